@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Throughput of the fused SignRot online path (rotate + sign-adjust + asymmetric INT4 quant).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 3]
+
+One step = one pass of the online path over the workload's T tokens resident in HBM
+(signrot_rotate_quant on [T, n] bf16 rows -> packed INT4 codes + fp32 scale/zero). The outlier
+channel and sign vector come from a calibration pass (signrot_calibrate + signrot_build_sign) run
+once before timing; its time is reported separately under "calibration". Multi-GPU runs shard
+tokens (weak scaling: every rank processes its own T tokens, no data-path collective).
+
+Rank 0 prints one JSON line. --impl reference times the float64 CPU oracle on a bounded sample
+of the same workload (the baseline this build is measured against).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from rotation_activation_quantization_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "tokens/s and achieved HBM GB/s (% of B200 peak) for fused rotate+INT4 quant"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=3, help="workload index (1..5); 3 = LLaMA3-8B down_proj")
+    ap.add_argument("--tokens", type=int, default=None, help="override tokens per GPU")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+def workload(args) -> syn.Workload:
+    w = syn.workload(args.config)
+    return w.with_T(args.tokens) if args.tokens else w
+
+
+def bytes_per_token(w: syn.Workload) -> int:
+    """Algorithmic HBM bytes per token: activations in, packed INT4 out, fp32 scale + zero."""
+    return w.in_bytes * w.n + w.n // 2 + 8
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return {"hbm_gbs": float(json.load(f)["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_sources_digest() -> str:
+    csrc = os.path.join(ROOT, "rotation_activation_quantization_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(w: syn.Workload, digest: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on these sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    e = rec.get(f"config{w.index}")
+    if not e or e.get("kernel_sources") != digest:
+        return None
+    return float(e["dram_bytes_per_token"]) * w.T
+
+
+def cpu_cores() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = max((i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"), default=0)
+        if n:
+            return int(n)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(w: syn.Workload, seconds: float, tokens_per_call: int = 8):
+    """Time the CPU oracle (float64 dense rotation + fp32 quantizer) on token blocks until the
+    budget is spent. Returns (tokens/s, tokens, seconds)."""
+    from oracle import signrot_oracle as o
+
+    d = syn.draw_d(w)
+    xc = o.to_f64(syn.draw_calibration(w, 0, min(256, syn.calibration_size(w))), w.dtype)
+    k, xk = o.calibrate(xc)
+    s = o.build_sign(w.n, k, xk, d)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        x = o.to_f64(syn.draw_tokens(w, done % w.T, done % w.T + tokens_per_call), w.dtype)
+        o.rotate_quant(x, d, s)
+        done += x.shape[0]
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return done / el, done, el
+
+
+class ClockSampler:
+    """Polls NVML (the source nvidia-smi reads) for SM clock, power and throttle reasons while
+    the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x10: "sync_boost", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz, self.err = [], 0, None, None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.nv = pynvml
+            self.max_mhz = self.nv.nvmlDeviceGetMaxClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+        except Exception as e:  # clocks are reported as unavailable, never invented
+            self.h, self.err = None, f"{type(e).__name__}: {e}"
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception as e:
+                self.err = f"{type(e).__name__}: {e}"
+                return
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.h is not None:
+            self._t.join(timeout=2)
+
+    def report(self) -> dict:
+        if self.h is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": self.err or "no samples"}
+        reasons = [name for bit, name in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def run_reference(args) -> int:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = workload(args)
+    cores = cpu_cores()
+    tokens_per_step = 4
+    from oracle import signrot_oracle as o
+
+    d = syn.draw_d(w)
+    xc = o.to_f64(syn.draw_calibration(w, 0, min(256, syn.calibration_size(w))), w.dtype)
+    k, xk = o.calibrate(xc)
+    s = o.build_sign(w.n, k, xk, d)
+    xs = o.to_f64(syn.draw_tokens(w, 0, tokens_per_step), w.dtype)
+    t0 = time.perf_counter()
+    for _ in range(max(args.warmup, 1) if args.warmup else 0):
+        o.rotate_quant(xs, d, s)
+    step_s = max((time.perf_counter() - t0) / max(args.warmup, 1), 1e-6)
+    budget = 150.0
+    steps = max(1, min(args.steps, int(budget / step_s)))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        o.rotate_quant(xs, d, s)
+    el = time.perf_counter() - t0
+    value = tokens_per_step * steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": steps, "steps_requested": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "n": w.n, "tokens_per_step": tokens_per_step,
+                   "input_dtype": w.dtype},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{tokens_per_step} tokens of {w.name} per step, dense float64 "
+                                   f"O(n^2) rotation + fp32 quantizer"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args) -> int:
+    import torch
+    import torch.distributed as dist
+
+    from rotation_activation_quantization_b200 import signrot as sr
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+    sr.lib()
+
+    w = workload(args)
+    T, n = w.T, w.n
+    # inputs: this rank's own T tokens (weak scaling), D, and the calibration batch
+    x_np = syn.draw_tokens(w, rank * T, (rank + 1) * T)
+    d_np = syn.draw_d(w)
+    xc_np = syn.draw_calibration(w)
+
+    def to_dev(a):
+        if w.dtype == "bf16":
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(a).to(dev)
+
+    x = to_dev(x_np)
+    d = torch.from_numpy(d_np).to(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # calibration (once per model; timed on its own)
+    xc = to_dev(xc_np)
+    ws = torch.empty(n, dtype=torch.int64, device=dev)
+    for _ in range(2):
+        k, xk, _ = sr.calibrate(xc, ws=ws)
+        s = sr.build_sign(n, k, xk, d)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    k, xk, _ = sr.calibrate(xc, ws=ws)
+    s = sr.build_sign(n, k, xk, d)
+    c1.record(stream)
+    torch.cuda.synchronize(dev)
+    calib_ms = c0.elapsed_time(c1)
+    del xc
+
+    q = torch.empty((T, n // 2), dtype=torch.uint8, device=dev)
+    scale = torch.empty(T, dtype=torch.float32, device=dev)
+    zero = torch.empty(T, dtype=torch.float32, device=dev)
+
+    def step():
+        sr.rotate_quant(x, d, s, q=q, scale=scale, zero=zero)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = sr.kernel_launches()
+    with sampler:
+        ev[0].record(stream)
+        for i in range(K):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+    launches = sr.kernel_launches() - launches0
+    if world > 1:
+        dist.barrier()
+    per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    region_ms = ev[0].elapsed_time(ev[K])
+    t = torch.tensor([region_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    region_ms_max = float(t.item())
+
+    # end to end through the same public call: pinned host -> HBM, rotate_quant, HBM -> pinned host
+    E = args.e2e_steps or max(3, min(K, 20))
+    xh = torch.from_numpy(x_np.view(np.int16) if w.dtype == "bf16" else x_np).pin_memory()
+    xe = torch.empty_like(x)
+    qh = torch.empty((T, n // 2), dtype=torch.uint8).pin_memory()
+    sh = torch.empty(T, dtype=torch.float32).pin_memory()
+    zh = torch.empty(T, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        xe.view(torch.int16 if w.dtype == "bf16" else torch.float32).copy_(xh, non_blocking=True)
+        sr.rotate_quant(xe, d, s, q=q, scale=scale, zero=zero)
+        qh.copy_(q, non_blocking=True)
+        sh.copy_(scale, non_blocking=True)
+        zh.copy_(zero, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_ms = float(te.item())
+    h2d = x.numel() * x.element_size()
+    d2h = q.numel() + 4 * scale.numel() + 4 * zero.numel()
+
+    if rank == 0:
+        bpt = bytes_per_token(w)
+        bytes_per_launch = bpt * T
+        avg_launch_ms = statistics.fmean(per_launch)
+        achieved = bytes_per_launch / (avg_launch_ms * 1e-3) / 1e9
+        peaks = measured_peaks()
+        digest = kernel_sources_digest()
+        traffic = recorded_traffic(w, digest)
+        value = world * T * K / (region_ms_max * 1e-3)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": region_ms_max / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {
+                "workload": w.name, "n": n, "tokens_per_gpu": T, "global_tokens": world * T,
+                "input_dtype": w.dtype, "output": "INT4 packed [T, n/2] + fp32 scale/zero [T]",
+                "parallelism": f"token-sharded x{world} (no collective)",
+                "l2": f"inputs larger than L2 ({bytes_per_launch / 1e6:.1f} MB per step vs "
+                      f"{L2_BYTES / 1e6:.0f} MB), no flush",
+            },
+            "hbm_gbs": achieved,
+            "hbm_frac": achieved / peaks["hbm_gbs"],
+            "roofline": {
+                "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "peak_source": peaks["source"], "bytes_per_token": bpt,
+                "kernel": "signrot_rotate_quant", "kernel_sources": digest,
+                "launch_ms_median": statistics.median(per_launch),
+            },
+            "e2e": {"value": world * T * E / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms / E, "steps": E},
+            "gpu_launches": int(launches),
+            "calibration": {"tokens": int(xc_np.shape[0]), "ms": calib_ms,
+                            "gbs": xc_np.shape[0] * n * w.in_bytes / (calib_ms * 1e-3) / 1e9},
+            "clocks": sampler.report(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, done, el = oracle_sample(w, args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                                    "sample": f"{done} tokens of {w.name} in {el:.1f} s (float64 dense "
+                                              f"O(n^2) rotation + fp32 quantizer)"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None) -> int:
+    args = parse(argv)
+    return run_reference(args) if args.impl == "reference" else run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,140 @@
+/*
+ * signrot.h -- C ABI of the SignRot online down-projection activation path on B200 (sm_100a).
+ *
+ * Per token row x in R^n (the input of a LLaMA MLP's down projection) the path computes
+ *
+ *     y = diag(s) . H . diag(D) . x / sqrt(n)                       (rotation + sign adjustment)
+ *     lo, hi = min_j y_j, max_j y_j
+ *     scale = (hi - lo) / 15,  zero = rne(-lo / scale)              (asymmetric per-token grid)
+ *     q_j = clamp(rne(y_j / scale) + zero, 0, 15)                   (INT4 codes, two per byte)
+ *
+ * Sources. "SignRot: LLM Quantization with Massive Outlier-Aware Sign-Adjusted Rotation" (arXiv
+ * 2611.16502, abstract): the randomized Hadamard rotation applied online at the down-projection
+ * input by the fast Walsh-Hadamard transform, the sign adjustment vector built from the massive
+ * outlier channel found in one calibration pass, and asymmetric activation quantization. "SignRot
+ * for 4-bit LLM quantization -- Sign-adjusted Hadamard rotation" (learnaivisually.com explainer),
+ * paragraphs "Picture the photographer" (16 levels from the token's smallest to largest value),
+ * "The standard fix is rotation" (entries +/-1/sqrt(n)), "SignRot asks one crowd to walk across
+ * the hall" (largest absolute calibration activation; per-output sign of the outlier's entry),
+ * "The flip alone does nothing for a symmetric quantizer" (asymmetric zero-point) and "Worked
+ * example" (steps are range/15, no clipping).
+ *
+ * H = H_F kron H_M with n = F * M, F in {1, 28}, M = 2^m, channel j = a * M + b. H_M is
+ * Sylvester's (H_M[b][e] = (-1)^popcount(b & e)); H_28 is Paley's construction I over
+ * GF(27) = GF(3)[t]/(t^3 + 2t + 1) (row 0 all +1, column 0 = (1, -1, ..., -1), see
+ * signrot_get_h28). Supported n: 2^m for 1 <= m <= 15, and 28 * 2^m for 0 <= m <= 10.
+ *
+ * Conventions shared by every call:
+ *   - Every call returns a signrot_status; nothing is thrown across the ABI.
+ *   - Tensors are caller-owned DEVICE pointers unless a parameter says host. The library
+ *     allocates no device memory.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*, NULL = legacy default stream)
+ *     and is asynchronous: a return of SIGNROT_OK means the launch was accepted. Device-side
+ *     faults surface on the caller's next synchronisation, as for any CUDA kernel.
+ *   - Activation rows are row-major: row t starts at element t * ld (ld >= n, in elements).
+ *   - T == 0 is a no-op that returns SIGNROT_OK.
+ *   - Inputs must be finite; a NaN or Inf in x gives unspecified codes (no fault).
+ */
+#ifndef SIGNROT_H
+#define SIGNROT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t signrot_status;
+#define SIGNROT_OK 0
+#define SIGNROT_ERR_INVALID_ARG 1   /* null pointer, negative size, ld < n, bad dtype, ... */
+#define SIGNROT_ERR_UNSUPPORTED_N 2 /* n not of the form 2^m or 28 * 2^m (see above)      */
+#define SIGNROT_ERR_ALIGNMENT 3     /* pointer not aligned to its element type            */
+#define SIGNROT_ERR_CUDA 4          /* a CUDA runtime call failed; see signrot_last_error */
+#define SIGNROT_ERR_UNSUPPORTED 5   /* e.g. bits != 4, clip outside (0, 1]                 */
+
+/* Storage type of the activations x. */
+#define SIGNROT_BF16 0
+#define SIGNROT_F32 1
+
+/*
+ * signrot_calibrate -- per-channel max |x| over calibration tokens, then the outlier channel.
+ *
+ * Follows the abstract's "single calibration forward pass" and the explainer's "finds the channel
+ * with the largest absolute activation". Reads x[T, n] (dtype, leading dimension ld) and folds it
+ * into the workspace ws[n] (uint64, device, caller-owned, 8 * n bytes), which keeps for every
+ * channel i the largest |x_{t,i}| seen, the first token index attaining it and that value's sign.
+ * Token indices are t_offset + t, so a calibration set streamed in chunks keeps "first token"
+ * global (0 <= t_offset, t_offset + T <= 2^31 - 1).
+ *   accumulate == 0: ws is reset first (this call starts a new calibration);
+ *   accumulate != 0: this chunk is folded into what ws already holds.
+ * After folding, writes k_out[0] (int32, device) = the lowest channel index attaining
+ * max_i max_t |x_{t,i}|, and xk_out[0] (float, device) = the signed value x_{t*,k} at the first
+ * token t* attaining it. T == 0 with accumulate != 0 only recomputes k and x_k from ws.
+ */
+signrot_status signrot_calibrate(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                 int64_t t_offset, uint64_t* ws, int32_t accumulate,
+                                 int32_t* k_out, float* xk_out, void* stream);
+
+/*
+ * signrot_build_sign -- the sign adjustment vector s.
+ *
+ * Follows the explainer's "SignRot asks one crowd to walk across the hall": every output j is
+ * multiplied by the sign of the outlier column's entry, so the outlier adds the same +|M|/sqrt(n)
+ * to every output. Here s_j = +1 if H[j][k] * D_k * x_k >= 0 else -1, with k = k[0] and
+ * x_k = xk[0] read on the device (as written by signrot_calibrate). d[n] and s_out[n] are int8
+ * +/-1, device. Passing x_k > 0 gives the literal "sign of that row's entry" form.
+ */
+signrot_status signrot_build_sign(int32_t n, const int32_t* k, const float* xk, const int8_t* d,
+                                  int8_t* s_out, void* stream);
+
+/*
+ * signrot_rotate -- the rotated, sign-adjusted rows in fp32 (the check path).
+ *
+ * y[t * ldy + j] = s_j * (H . diag(D) . x_t)_j / sqrt(n) for t < T, j < n. d[n] int8 +/-1;
+ * s[n] int8 +/-1 or NULL (all +1); y float, device, ldy >= n. Follows "The standard fix is
+ * rotation" (entries +/-1/sqrt(n), every output a signed sum of all inputs) and the abstract's
+ * fast Walsh-Hadamard transform.
+ */
+signrot_status signrot_rotate(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                              const int8_t* d, const int8_t* s, float* y, int64_t ldy,
+                              void* stream);
+
+/*
+ * signrot_rotate_quant -- the fused online path: rotate, sign-adjust, quantize to packed INT4.
+ *
+ * For each row t: y as in signrot_rotate, then with c = clip, lo = c * min y, hi = c * max y:
+ *   scale[t] = (hi - lo) / 15, zero[t] = rne(-lo / scale[t])   (fp32; zero is integer-valued and
+ *   usually far outside [0, 15], which is why it is stored as fp32)
+ *   code_j = clamp(rne(y_j / scale[t]) + zero[t], 0, 15)       (rne: nearest, ties to even)
+ *   a row with hi == lo gets scale = 1, zero = rne(-lo).
+ * q[t * (n / 2) + i] = code_{2i} | code_{2i+1} << 4 (uint8, device, [T, n/2] row-major; n even).
+ * Dequantize with (code - zero) * scale. bits must be 4; clip in (0, 1] (1 = no clipping, as in
+ * the worked example). s may be NULL (plain rotation, no sign adjustment).
+ * The codes are decided in fp32 with the reciprocal of the scale, so a code may differ by one
+ * from the formula above where y / scale lies within an ulp of a half-integer.
+ */
+signrot_status signrot_rotate_quant(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                    const int8_t* d, const int8_t* s, int32_t bits, float clip,
+                                    uint8_t* q, float* scale, float* zero, void* stream);
+
+/* Host: writes H_28 (Paley, GF(27), the orientation described above) row-major into out[784]. */
+signrot_status signrot_get_h28(int8_t* out);
+
+/* 1 if n is a supported row length, else 0. */
+int32_t signrot_supported_n(int32_t n);
+
+/* Static English text for a status code. */
+const char* signrot_status_string(signrot_status status);
+
+/* Details of the last failure on the calling host thread ("" if none). */
+const char* signrot_last_error(void);
+
+/* Number of kernels this library has launched in this process (all threads, all devices). */
+uint64_t signrot_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SIGNROT_H */

@@ -201,7 +201,7 @@ def factor_n(n: int) -> tuple[int, int]:
     raise ValueError(f"unsupported n = {n}")
 
 
-@lru_cache(maxsize=4)
+@lru_cache(maxsize=2)
 def hadamard(n: int) -> np.ndarray:
     """Dense H_n = H_F kron H_M as int8 [n, n] (unnormalised, entries +/-1)."""
     F, M = factor_n(n)

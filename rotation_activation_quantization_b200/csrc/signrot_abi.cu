@@ -1,0 +1,234 @@
+// The C ABI (include/signrot.h): argument validation, shape factorisation, dispatch to the
+// kernels, and error reporting. No device memory is allocated here.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <atomic>
+
+#include <cuda_runtime.h>
+
+#include "signrot.h"
+#include "signrot_internal.h"
+
+namespace signrot {
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+}  // namespace signrot
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+signrot_status fail(signrot_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+signrot_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SIGNROT_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool factor_n(int32_t n, signrot::Shape* sh) {
+  if (n <= 0) return false;
+  const auto pow2 = [](int32_t v) { return v > 0 && (v & (v - 1)) == 0; };
+  const auto lg = [](int32_t v) {
+    int m = 0;
+    while ((1 << m) < v) ++m;
+    return m;
+  };
+  if (pow2(n) && n >= 2 && n <= (1 << 15)) {
+    *sh = {n, 1, lg(n)};
+    return true;
+  }
+  if (n % 28 == 0 && pow2(n / 28) && n / 28 <= (1 << 10)) {
+    *sh = {n, 28, lg(n / 28)};
+    return true;
+  }
+  return false;
+}
+
+struct H28State {
+  int8_t h[28][28];
+  signrot::H28Masks masks;
+};
+
+const H28State& h28_state() {
+  static H28State st;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    signrot::paley_h28(st.h);
+    for (int a = 0; a < 28; ++a) {
+      uint32_t m = 0;
+      for (int c = 0; c < 28; ++c)
+        if (st.h[a][c] < 0) m |= 1u << c;
+      st.masks.row[a] = m;
+    }
+  });
+  return st;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+signrot_status check_rows(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                          signrot::Shape* sh) {
+  if (dtype != SIGNROT_BF16 && dtype != SIGNROT_F32)
+    return fail(SIGNROT_ERR_INVALID_ARG, "dtype %d is neither SIGNROT_BF16 nor SIGNROT_F32", dtype);
+  if (T < 0) return fail(SIGNROT_ERR_INVALID_ARG, "T = %lld < 0", static_cast<long long>(T));
+  if (!factor_n(n, sh))
+    return fail(SIGNROT_ERR_UNSUPPORTED_N, "n = %d is not 2^m (1<=m<=15) or 28*2^m (0<=m<=10)", n);
+  if (ld < n) return fail(SIGNROT_ERR_INVALID_ARG, "ld = %lld < n = %d", static_cast<long long>(ld), n);
+  if (T > 0 && x == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "x is NULL");
+  if (!aligned(x, dtype == SIGNROT_BF16 ? 2 : 4))
+    return fail(SIGNROT_ERR_ALIGNMENT, "x is not aligned to its element size");
+  return SIGNROT_OK;
+}
+
+signrot_status run_rotate(signrot::RotateArgs& a, cudaStream_t st) {
+  const auto& h = h28_state().masks;
+  a.inv_sqrt_n = static_cast<float>(1.0 / std::sqrt(static_cast<double>(a.shape.n)));
+  cudaError_t e = signrot::launch_rotate_fast(a, h, st);
+  if (e == cudaErrorNotSupported) {
+    (void)cudaGetLastError();
+    e = signrot::launch_rotate_generic(a, h, st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "rotate launch");
+  return SIGNROT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+signrot_status signrot_calibrate(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                 int64_t t_offset, uint64_t* ws, int32_t accumulate,
+                                 int32_t* k_out, float* xk_out, void* stream) {
+  g_last_error[0] = '\0';
+  signrot::Shape sh;
+  signrot_status st = check_rows(x, dtype, T, n, ld, &sh);
+  if (st != SIGNROT_OK) return st;
+  if (ws == nullptr || k_out == nullptr || xk_out == nullptr)
+    return fail(SIGNROT_ERR_INVALID_ARG, "ws, k_out and xk_out must be device pointers");
+  if (!aligned(ws, 8) || !aligned(k_out, 4) || !aligned(xk_out, 4))
+    return fail(SIGNROT_ERR_ALIGNMENT, "ws (8 B), k_out and xk_out (4 B) misaligned");
+  if (t_offset < 0 || t_offset + T > 0x7fffffffLL)
+    return fail(SIGNROT_ERR_INVALID_ARG, "token indices t_offset + t must stay below 2^31 - 1");
+  auto s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (!accumulate) {
+    e = cudaMemsetAsync(ws, 0, sizeof(uint64_t) * static_cast<size_t>(n), s);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
+  }
+  signrot::CalibArgs a{x, dtype, T, n, ld, t_offset, reinterpret_cast<unsigned long long*>(ws)};
+  if ((e = signrot::launch_calibrate_fold(a, s)) != cudaSuccess) return cuda_fail(e, "calibrate fold");
+  e = signrot::launch_calibrate_argmax(reinterpret_cast<const unsigned long long*>(ws), n, k_out, xk_out, s);
+  if (e != cudaSuccess) return cuda_fail(e, "calibrate argmax");
+  return SIGNROT_OK;
+}
+
+signrot_status signrot_build_sign(int32_t n, const int32_t* k, const float* xk, const int8_t* d,
+                                  int8_t* s_out, void* stream) {
+  g_last_error[0] = '\0';
+  signrot::Shape sh;
+  if (!factor_n(n, &sh))
+    return fail(SIGNROT_ERR_UNSUPPORTED_N, "n = %d is not 2^m (1<=m<=15) or 28*2^m (0<=m<=10)", n);
+  if (k == nullptr || xk == nullptr || d == nullptr || s_out == nullptr)
+    return fail(SIGNROT_ERR_INVALID_ARG, "k, xk, d and s_out must be device pointers");
+  if (!aligned(k, 4) || !aligned(xk, 4)) return fail(SIGNROT_ERR_ALIGNMENT, "k or xk misaligned");
+  cudaError_t e = signrot::launch_build_sign(sh, k, xk, d, s_out, h28_state().masks,
+                                             static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "build_sign launch");
+  return SIGNROT_OK;
+}
+
+signrot_status signrot_rotate(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                              const int8_t* d, const int8_t* s, float* y, int64_t ldy,
+                              void* stream) {
+  g_last_error[0] = '\0';
+  signrot::Shape sh;
+  signrot_status st = check_rows(x, dtype, T, n, ld, &sh);
+  if (st != SIGNROT_OK) return st;
+  if (d == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "d is NULL");
+  if (T > 0 && y == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < n) return fail(SIGNROT_ERR_INVALID_ARG, "ldy < n");
+  if (!aligned(y, 4)) return fail(SIGNROT_ERR_ALIGNMENT, "y is not 4-byte aligned");
+  if (T == 0) return SIGNROT_OK;
+  signrot::RotateArgs a{};
+  a.x = x;
+  a.dtype = dtype;
+  a.T = T;
+  a.ld = ld;
+  a.shape = sh;
+  a.d = d;
+  a.s = s;
+  a.y = y;
+  a.ldy = ldy;
+  a.clip = 1.f;
+  return run_rotate(a, static_cast<cudaStream_t>(stream));
+}
+
+signrot_status signrot_rotate_quant(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                    const int8_t* d, const int8_t* s, int32_t bits, float clip,
+                                    uint8_t* q, float* scale, float* zero, void* stream) {
+  g_last_error[0] = '\0';
+  signrot::Shape sh;
+  signrot_status st = check_rows(x, dtype, T, n, ld, &sh);
+  if (st != SIGNROT_OK) return st;
+  if (bits != 4) return fail(SIGNROT_ERR_UNSUPPORTED, "bits = %d; only 4 is supported", bits);
+  if (!(clip > 0.f && clip <= 1.f)) return fail(SIGNROT_ERR_UNSUPPORTED, "clip must lie in (0, 1]");
+  if (d == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "d is NULL");
+  if (T > 0 && (q == nullptr || scale == nullptr || zero == nullptr))
+    return fail(SIGNROT_ERR_INVALID_ARG, "q, scale and zero must be device pointers");
+  if (!aligned(scale, 4) || !aligned(zero, 4))
+    return fail(SIGNROT_ERR_ALIGNMENT, "scale / zero not 4-byte aligned");
+  if (T == 0) return SIGNROT_OK;
+  signrot::RotateArgs a{};
+  a.x = x;
+  a.dtype = dtype;
+  a.T = T;
+  a.ld = ld;
+  a.shape = sh;
+  a.d = d;
+  a.s = s;
+  a.q = q;
+  a.scale = scale;
+  a.zero = zero;
+  a.clip = clip;
+  return run_rotate(a, static_cast<cudaStream_t>(stream));
+}
+
+signrot_status signrot_get_h28(int8_t* out) {
+  if (out == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "out is NULL");
+  std::memcpy(out, h28_state().h, 28 * 28);
+  return SIGNROT_OK;
+}
+
+int32_t signrot_supported_n(int32_t n) {
+  signrot::Shape sh;
+  return factor_n(n, &sh) ? 1 : 0;
+}
+
+const char* signrot_status_string(signrot_status status) {
+  switch (status) {
+    case SIGNROT_OK: return "ok";
+    case SIGNROT_ERR_INVALID_ARG: return "invalid argument";
+    case SIGNROT_ERR_UNSUPPORTED_N: return "unsupported row length n";
+    case SIGNROT_ERR_ALIGNMENT: return "misaligned pointer";
+    case SIGNROT_ERR_CUDA: return "CUDA runtime error";
+    case SIGNROT_ERR_UNSUPPORTED: return "unsupported option";
+    default: return "unknown status";
+  }
+}
+
+const char* signrot_last_error(void) { return g_last_error; }
+
+uint64_t signrot_kernel_launches(void) { return signrot::g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

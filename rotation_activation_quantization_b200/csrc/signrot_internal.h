@@ -1,0 +1,72 @@
+// Internal launch interface between the C ABI (signrot_abi.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace signrot {
+
+// Counts every kernel launch the library issues (read by signrot_kernel_launches).
+void count_launch(int n = 1);
+
+// Library-owned Paley H_28 (paley_gf27.cpp), row-major, entries +/-1.
+void paley_h28(int8_t h[28][28]);
+
+// H_28 as sign masks: bit c of row[a] is set iff H_28[a][c] == -1. Passed by value in kernel
+// parameters (constant bank), so no per-device state has to be initialised.
+struct H28Masks {
+  uint32_t row[28];
+};
+
+enum : int32_t { kBF16 = 0, kF32 = 1 };
+
+// n = F * 2^logM, F in {1, 28}.
+struct Shape {
+  int32_t n;
+  int32_t F;
+  int32_t logM;
+};
+
+struct RotateArgs {
+  const void* x;
+  int32_t dtype;
+  int64_t T;
+  int64_t ld;
+  Shape shape;
+  const int8_t* d;  // [n] +/-1
+  const int8_t* s;  // [n] +/-1 or null
+  // check path (fp32 y) -- y != null
+  float* y;
+  int64_t ldy;
+  // quantized path -- q != null
+  uint8_t* q;
+  float* scale;
+  float* zero;
+  float clip;
+  float inv_sqrt_n;  // fp32(1 / sqrt(n))
+};
+
+// Generic row kernel: any supported n, any element-aligned x. One CTA per row (grid-stride).
+cudaError_t launch_rotate_generic(const RotateArgs& a, const H28Masks& h, cudaStream_t st);
+
+// Fast fused kernels for the shapes they cover; return cudaErrorNotSupported when the shape or
+// the alignment is not theirs (the caller then uses the generic kernel).
+cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStream_t st);
+
+struct CalibArgs {
+  const void* x;
+  int32_t dtype;
+  int64_t T;
+  int32_t n;
+  int64_t ld;
+  int64_t t_offset;
+  unsigned long long* ws;
+};
+cudaError_t launch_calibrate_fold(const CalibArgs& a, cudaStream_t st);
+cudaError_t launch_calibrate_argmax(const unsigned long long* ws, int32_t n, int32_t* k_out,
+                                    float* xk_out, cudaStream_t st);
+cudaError_t launch_build_sign(Shape shape, const int32_t* k, const float* xk, const int8_t* d,
+                              int8_t* s_out, const H28Masks& h, cudaStream_t st);
+
+}  // namespace signrot

@@ -1,0 +1,191 @@
+"""Python binding of the SignRot C ABI (include/signrot.h): argument marshalling only.
+
+Every step of the path runs in the CUDA library ``lib/libsignrot.so``; this module checks tensor
+placement, dtypes and strides, allocates outputs with torch when the caller does not pass them,
+and forwards raw device pointers and the current CUDA stream. There is no CPU fallback: if the
+library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libsignrot.so")
+_lib = None
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_N, ERR_ALIGNMENT, ERR_CUDA, ERR_UNSUPPORTED = range(6)
+BF16, F32 = 0, 1
+
+_c_i32, _c_i64, _c_p, _c_f = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_float
+
+_SIGNATURES = {
+    "signrot_calibrate": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_i64, _c_p, _c_i32, _c_p, _c_p, _c_p],
+    "signrot_build_sign": [_c_i32, _c_p, _c_p, _c_p, _c_p, _c_p],
+    "signrot_rotate": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_i64, _c_p],
+    "signrot_rotate_quant": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_i32, _c_f,
+                             _c_p, _c_p, _c_p, _c_p],
+    "signrot_get_h28": [_c_p],
+    "signrot_supported_n": [_c_i32],
+    "signrot_status_string": [_c_i32],
+    "signrot_last_error": [],
+    "signrot_kernel_launches": [],
+}
+
+EXPORTED = tuple(_SIGNATURES)
+
+
+class SignRotError(RuntimeError):
+    def __init__(self, fn: str, status: int, detail: str):
+        super().__init__(f"{fn} failed with status {status}: {detail}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsignrot.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m rotation_activation_quantization_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        for name, args in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int32
+        L.signrot_status_string.restype = ctypes.c_char_p
+        L.signrot_last_error.restype = ctypes.c_char_p
+        L.signrot_kernel_launches.restype = ctypes.c_uint64
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != OK:
+        L = lib()
+        detail = L.signrot_last_error().decode() or L.signrot_status_string(status).decode()
+        raise SignRotError(fn, status, detail)
+
+
+def _dtype_code(x: torch.Tensor) -> int:
+    if x.dtype == torch.bfloat16:
+        return BF16
+    if x.dtype == torch.float32:
+        return F32
+    raise TypeError(f"activations must be bfloat16 or float32, got {x.dtype}")
+
+
+def _rows(x: torch.Tensor) -> tuple[int, int, int]:
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D [T, n] tensor with unit stride along n")
+    if not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor")
+    return x.shape[0], x.shape[1], x.stride(0) if x.shape[0] > 1 else x.shape[1]
+
+
+def _stream(dev: torch.device, stream) -> int:
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, dev, dtype, numel, name):
+    if t.device != dev or t.dtype != dtype or t.numel() < numel or not t.is_contiguous():
+        raise ValueError(f"{name}: need a contiguous {dtype} tensor with >= {numel} elements on {dev}")
+
+
+def kernel_launches() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(lib().signrot_kernel_launches())
+
+
+def supported_n(n: int) -> bool:
+    return bool(lib().signrot_supported_n(int(n)))
+
+
+def get_h28() -> np.ndarray:
+    out = np.zeros(28 * 28, dtype=np.int8)
+    _check("signrot_get_h28", lib().signrot_get_h28(out.ctypes.data))
+    return out.reshape(28, 28)
+
+
+def calibrate(x: torch.Tensor, ws: torch.Tensor | None = None, accumulate: bool = False,
+              t_offset: int = 0, k_out: torch.Tensor | None = None,
+              xk_out: torch.Tensor | None = None, stream=None):
+    """Fold calibration rows x [T, n] into ws [n] (int64 storage of the uint64 keys) and return
+    (k, x_k) as 1-element device tensors (int32, float32). Returns (k, x_k, ws)."""
+    T, n, ld = _rows(x)
+    dev = x.device
+    ws = torch.empty(n, dtype=torch.int64, device=dev) if ws is None else ws
+    _need(ws, dev, torch.int64, n, "ws")
+    k_out = torch.empty(1, dtype=torch.int32, device=dev) if k_out is None else k_out
+    xk_out = torch.empty(1, dtype=torch.float32, device=dev) if xk_out is None else xk_out
+    with torch.cuda.device(dev):
+        st = lib().signrot_calibrate(_ptr(x), _dtype_code(x), T, n, ld, int(t_offset), _ptr(ws),
+                                     int(bool(accumulate)), _ptr(k_out), _ptr(xk_out), _stream(dev, stream))
+    _check("signrot_calibrate", st)
+    return k_out, xk_out, ws
+
+
+def build_sign(n: int, k: torch.Tensor, xk: torch.Tensor, d: torch.Tensor,
+               s_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    dev = d.device
+    _need(d, dev, torch.int8, n, "d")
+    _need(k, dev, torch.int32, 1, "k")
+    _need(xk, dev, torch.float32, 1, "xk")
+    s_out = torch.empty(n, dtype=torch.int8, device=dev) if s_out is None else s_out
+    _need(s_out, dev, torch.int8, n, "s_out")
+    with torch.cuda.device(dev):
+        st = lib().signrot_build_sign(int(n), _ptr(k), _ptr(xk), _ptr(d), _ptr(s_out), _stream(dev, stream))
+    _check("signrot_build_sign", st)
+    return s_out
+
+
+def rotate(x: torch.Tensor, d: torch.Tensor, s: torch.Tensor | None = None,
+           out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """fp32 y = s (.) H D x / sqrt(n) for every row of x [T, n]."""
+    T, n, ld = _rows(x)
+    dev = x.device
+    _need(d, dev, torch.int8, n, "d")
+    if s is not None:
+        _need(s, dev, torch.int8, n, "s")
+    out = torch.empty((T, n), dtype=torch.float32, device=dev) if out is None else out
+    if out.shape != (T, n) or out.stride(1) != 1 or out.dtype != torch.float32 or out.device != dev:
+        raise ValueError("out must be a float32 [T, n] tensor with unit stride along n on x's device")
+    ldy = out.stride(0) if T > 1 else n
+    with torch.cuda.device(dev):
+        st = lib().signrot_rotate(_ptr(x), _dtype_code(x), T, n, ld, _ptr(d), _ptr(s), _ptr(out), ldy,
+                                  _stream(dev, stream))
+    _check("signrot_rotate", st)
+    return out
+
+
+def rotate_quant(x: torch.Tensor, d: torch.Tensor, s: torch.Tensor | None = None, bits: int = 4,
+                 clip: float = 1.0, q: torch.Tensor | None = None, scale: torch.Tensor | None = None,
+                 zero: torch.Tensor | None = None, stream=None):
+    """The fused path: returns (q uint8 [T, n/2], scale f32 [T], zero f32 [T])."""
+    T, n, ld = _rows(x)
+    dev = x.device
+    _need(d, dev, torch.int8, n, "d")
+    if s is not None:
+        _need(s, dev, torch.int8, n, "s")
+    q = torch.empty((T, n // 2), dtype=torch.uint8, device=dev) if q is None else q
+    scale = torch.empty(T, dtype=torch.float32, device=dev) if scale is None else scale
+    zero = torch.empty(T, dtype=torch.float32, device=dev) if zero is None else zero
+    _need(q, dev, torch.uint8, T * (n // 2), "q")
+    _need(scale, dev, torch.float32, T, "scale")
+    _need(zero, dev, torch.float32, T, "zero")
+    with torch.cuda.device(dev):
+        st = lib().signrot_rotate_quant(_ptr(x), _dtype_code(x), T, n, ld, _ptr(d), _ptr(s), int(bits),
+                                        float(clip), _ptr(q), _ptr(scale), _ptr(zero), _stream(dev, stream))
+    _check("signrot_rotate_quant", st)
+    return q, scale, zero

@@ -161,3 +161,26 @@ def draw_calibration(w: Workload, t0: int = 0, t1: int | None = None) -> np.ndar
 
 def calibration_size(w: Workload) -> int:
     return w.calib_T if w.calib_T else w.T
+
+
+def random_rows(n: int, T: int, dtype: str = "bf16", seed: int = 0, outlier: float = 1500.0,
+                k: int | None = None, sigma: float = 0.3, base: str = "laplace",
+                outlier_sign: str = "random") -> tuple[np.ndarray, np.ndarray, int]:
+    """Small seeded rows for parity sweeps: ordinary channels plus one massive-outlier channel.
+
+    Returns (x encoded as bf16 bits or fp32, D as int8 +/-1, outlier channel k)."""
+    rng = _rng(7919, seed, n, T)
+    k = int(rng.integers(n)) if k is None else int(k)
+    if base == "laplace":
+        v = rng.laplace(0.0, sigma, size=(T, n))
+    else:
+        v = rng.normal(0.0, sigma, size=(T, n))
+    if outlier:
+        if outlier_sign == "random":
+            sgn = np.where(rng.random(T) < 0.5, -1.0, 1.0)
+        else:
+            sgn = np.full(T, 1.0 if outlier_sign == "+" else -1.0)
+        v[:, k] = sgn * rng.uniform(0.5 * outlier, outlier, size=T)
+    d = np.where(rng.random(n) < 0.5, -1, 1).astype(np.int8)
+    a32 = v.astype(np.float32)
+    return (f32_to_bf16_bits(a32) if dtype == "bf16" else a32), d, k
