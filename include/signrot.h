@@ -118,6 +118,52 @@ signrot_status signrot_rotate_quant(const void* x, int32_t dtype, int64_t T, int
                                     const int8_t* d, const int8_t* s, int32_t bits, float clip,
                                     uint8_t* q, float* scale, float* zero, void* stream);
 
+/*
+ * signrot_rotate_outlier / signrot_rotate_quant_outlier -- the same two calls with the sign
+ * adjustment given by its outlier channel instead of a materialised s: k[0] (int32, device) and
+ * x_k = xk[0] (float, device), as written by signrot_calibrate. The result equals calling
+ * signrot_rotate(_quant) with s = signrot_build_sign(n, k, xk, d) (bit for bit on the fused
+ * kernel). Because s_j = sgn(H[j][k] D_k x_k) is a signed column of H, it factorises along the
+ * Kronecker structure and is folded into the rotation itself, so the sign adjustment costs no
+ * per-element work (the explainer's "at inference the only new work is an element-wise sign
+ * flip", taken to zero). x_k == 0 means s = +1 everywhere.
+ */
+signrot_status signrot_rotate_outlier(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                      const int8_t* d, const int32_t* k, const float* xk, float* y,
+                                      int64_t ldy, void* stream);
+signrot_status signrot_rotate_quant_outlier(const void* x, int32_t dtype, int64_t T, int32_t n,
+                                            int64_t ld, const int8_t* d, const int32_t* k,
+                                            const float* xk, int32_t bits, float clip, uint8_t* q,
+                                            float* scale, float* zero, void* stream);
+
+/*
+ * signrot_rotate_quant_host -- the fused path between HOST buffers: x_host [T, ld] (pinned for
+ * overlap; pageable works but serialises) -> q_host [T, n/2], scale_host [T], zero_host [T].
+ * d (device, [n]) as above; the sign adjustment is s (device [n], or NULL) or, when k and xk
+ * (device) are both given, the outlier channel (then s must be NULL). The rows are streamed
+ * through the caller's device workspace in chunks: each chunk's host-to-device copy, kernel and
+ * device-to-host copy are enqueued on one of two library streams (created once per device), so
+ * copies in both directions overlap the neighbouring chunks. workspace must hold at least
+ * 2 * signrot_host_bytes_per_token(n, dtype) bytes (16-byte aligned); the chunk length is what
+ * fits in half of it. The caller's stream waits for all of it before its next work; the host
+ * outputs are complete once that stream is synchronised.
+ */
+signrot_status signrot_rotate_quant_host(const void* x_host, int32_t dtype, int64_t T, int32_t n,
+                                         int64_t ld, const int8_t* d, const int8_t* s,
+                                         const int32_t* k, const float* xk, int32_t bits, float clip,
+                                         uint8_t* q_host, float* scale_host, float* zero_host,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Device workspace bytes one token needs in signrot_rotate_quant_host (input row + outputs). */
+size_t signrot_host_bytes_per_token(int32_t n, int32_t dtype);
+
+/*
+ * Host, synchronous: writes the device error word of the current device to *code (0 = none;
+ * bit 0 = a fused kernel's bounded wait on its own pipeline expired and the kernel stopped
+ * early, leaving its outputs incomplete) and clears it when clear != 0.
+ */
+signrot_status signrot_device_error(int32_t* code, int32_t clear);
+
 /* Host: writes H_28 (Paley, GF(27), the orientation described above) row-major into out[784]. */
 signrot_status signrot_get_h28(int8_t* out);
 

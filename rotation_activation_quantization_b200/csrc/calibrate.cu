@@ -99,6 +99,10 @@ __global__ void build_sign_kernel(Shape sh, const int32_t* __restrict__ kp, cons
   if (j >= sh.n) return;
   const int k = *kp;
   const float xk = *xkp;
+  if (k < 0 || k >= sh.n) {  // not a channel index: no sign adjustment
+    s[j] = 1;
+    return;
+  }
   const int M1 = (1 << sh.logM) - 1;
   const int a = j >> sh.logM, b = j & M1;
   const int c = k >> sh.logM, e = k & M1;

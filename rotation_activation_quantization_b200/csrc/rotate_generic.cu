@@ -1,14 +1,18 @@
 // Generic rotate / rotate+quantize kernel: one CTA per token row, the row staged in shared
-// memory as fp32. Covers every supported n and any element-aligned input; the fused fast
-// kernels (rotate_fast.cu) take the shapes they are built for.
+// memory. Covers every supported n, fp32 or bf16 input and any element-aligned rows; the fused
+// tensor-core kernel (rotate_tc.cu) takes the bf16 shapes it is built for.
 //
 // Per row (SignRot explainer, "The standard fix is rotation" and "SignRot asks one crowd to walk
 // across the hall"; abstract: fast Walsh-Hadamard transform):
 //   1. x' = D (.) x                 (exact sign flips)
 //   2. H_28 across the stride-M axis (dense 28 x 28 block, F = 28 only)
 //   3. FWHT of length M along the contiguous axis, radix-2 stages
-//   4. y = s (.) w * fp32(1/sqrt(n))
+//   4. y = s (.) w / sqrt(n), rounded once to fp32
 //   5. check path: store y; quantized path: row min/max, scale, zero, codes, nibble pack.
+// The rotation accumulates in fp64 (fp32 only for n = 32768, whose fp64 row would not fit in
+// shared memory), so y is the correctly rounded fp32 of the exact rotation up to a rare double
+// rounding, and the quantizer then takes the same fp32 steps as the formula in the header
+// (true divisions, ties to even). This path is the slow, exact-decision reference on the device.
 #include <cstdint>
 
 #include "signrot_internal.h"
@@ -19,33 +23,51 @@ namespace {
 
 constexpr int kThreads = 512;
 
-template <typename Tin, bool kQuant>
-__global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, H28Masks h) {
-  extern __shared__ float buf[];
+template <typename Acc>
+__device__ __forceinline__ Acc neg_if(Acc v, bool neg) {
+  return neg ? -v : v;
+}
+
+template <typename Tin, typename Acc, bool kQuant>
+__global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, H28Masks h, double sqrt_n) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  Acc* buf = reinterpret_cast<Acc*>(smem_raw);
+  float* ybuf = reinterpret_cast<float*>(smem_raw);  // fp32 y, aliases buf after step 4
   __shared__ float red[64];
   const int n = a.shape.n;
   const int logM = a.shape.logM;
   const int M = 1 << logM;
   const Tin* __restrict__ x = static_cast<const Tin*>(a.x);
+  // sign vector from the outlier channel: s_j = sgn(H[j,k] D_k x_k), +1 everywhere if x_k = 0
+  bool pattern = false;
+  int c_k = 0, e_k = 0, sig_neg = 0;
+  if (a.kp != nullptr) {
+    const int k = *a.kp;
+    const float xk = *a.xkp;
+    pattern = xk != 0.f && k >= 0 && k < n;  // an out-of-range k applies no sign adjustment
+    if (pattern) {
+      c_k = k >> logM;
+      e_k = k & (M - 1);
+      sig_neg = ((xk < 0.f) != (a.d[k] < 0)) ? 1 : 0;
+    }
+  }
 
   for (int64_t t = blockIdx.x; t < a.T; t += gridDim.x) {
     const Tin* xr = x + t * a.ld;
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-      float v = load_as_float(xr + j);
-      buf[j] = a.d[j] < 0 ? -v : v;
-    }
+    for (int j = threadIdx.x; j < n; j += blockDim.x)
+      buf[j] = neg_if(static_cast<Acc>(load_as_float(xr + j)), a.d[j] < 0);
     __syncthreads();
 
     if (a.shape.F == 28) {
       for (int b = threadIdx.x; b < M; b += blockDim.x) {
-        float v[28];
+        Acc v[28];
 #pragma unroll
         for (int c = 0; c < 28; ++c) v[c] = buf[c * M + b];
         for (int r = 0; r < 28; ++r) {
           const uint32_t m = h.row[r];
-          float acc = 0.f;
+          Acc acc = 0;
 #pragma unroll
-          for (int c = 0; c < 28; ++c) acc += ((m >> c) & 1u) ? -v[c] : v[c];
+          for (int c = 0; c < 28; ++c) acc += neg_if(v[c], (m >> c) & 1u);
           buf[r * M + b] = acc;
         }
       }
@@ -57,38 +79,63 @@ __global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, 
         const int row = p >> (logM - 1);
         const int r = p & ((M >> 1) - 1);
         const int i = ((r & ~(hs - 1)) << 1) | (r & (hs - 1));
-        float* base = buf + row * M;
-        const float u = base[i], v = base[i + hs];
+        Acc* base = buf + row * M;
+        const Acc u = base[i], v = base[i + hs];
         base[i] = u + v;
         base[i + hs] = u - v;
       }
       __syncthreads();
     }
 
-    float lo = __int_as_float(0x7f800000), hi = -lo;
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-      float w = buf[j];
-      if (a.s != nullptr && a.s[j] < 0) w = -w;
-      const float yv = w * a.inv_sqrt_n;
-      if (kQuant) {
-        buf[j] = yv;
-        lo = fminf(lo, yv);
-        hi = fmaxf(hi, yv);
-      } else {
-        a.y[t * a.ldy + j] = yv;
+    // y in fp32: one rounding of s_j * w_j / sqrt(n)
+    float lo = pos_inf(), hi = -pos_inf();
+    constexpr int kPer = (sizeof(Acc) + sizeof(float) - 1) / sizeof(float);  // y overwrites buf in place
+    for (int j0 = 0; j0 < n; j0 += blockDim.x * kPer) {
+      float yv[kPer];
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) {
+        const int j = j0 + threadIdx.x * kPer + e;
+        yv[e] = 0.f;
+        if (j < n) {
+          bool neg;
+          if (pattern) {
+            neg = ((__popc((j & (M - 1)) & e_k) & 1) ^ sig_neg) != 0;
+            if (a.shape.F == 28) neg ^= ((h.row[j >> logM] >> c_k) & 1u) != 0;
+          } else {
+            neg = a.s != nullptr && a.s[j] < 0;
+          }
+          const Acc w = neg_if(buf[j], neg);
+          yv[e] = sizeof(Acc) == 8 ? static_cast<float>(static_cast<double>(w) / sqrt_n)
+                                   : static_cast<float>(w) * a.inv_sqrt_n;
+        }
       }
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) {
+        const int j = j0 + threadIdx.x * kPer + e;
+        if (j < n) {
+          if (kQuant) {
+            ybuf[j] = yv[e];
+            lo = fminf(lo, yv[e]);
+            hi = fmaxf(hi, yv[e]);
+          } else {
+            a.y[t * a.ldy + j] = yv[e];
+          }
+        }
+      }
+      __syncthreads();
     }
     if (kQuant) {
       block_minmax(lo, hi, red);
-      QuantGrid g = make_grid(lo, hi, a.clip);
+      const QuantGrid g = make_grid(lo, hi, a.clip);
       if (threadIdx.x == 0) {
         a.scale[t] = g.scale;
         a.zero[t] = g.zero;
       }
       uint8_t* qr = a.q + t * (n >> 1);
       for (int i = threadIdx.x; i < (n >> 1); i += blockDim.x) {
-        const uint32_t c0 = quant_code(buf[2 * i], g);
-        const uint32_t c1 = quant_code(buf[2 * i + 1], g);
+        const uint32_t c0 = quant_code_div(ybuf[2 * i], g);
+        const uint32_t c1 = quant_code_div(ybuf[2 * i + 1], g);
         qr[i] = static_cast<uint8_t>(c0 | (c1 << 4));
       }
     }
@@ -96,10 +143,10 @@ __global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, 
   }
 }
 
-template <typename Tin, bool kQuant>
+template <typename Tin, typename Acc, bool kQuant>
 cudaError_t launch_typed(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(a.shape.n) * sizeof(float);
-  auto kern = rotate_generic_kernel<Tin, kQuant>;
+  const size_t smem = static_cast<size_t>(a.shape.n) * sizeof(Acc);
+  auto kern = rotate_generic_kernel<Tin, Acc, kQuant>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -110,18 +157,23 @@ cudaError_t launch_typed(const RotateArgs& a, const H28Masks& h, cudaStream_t st
     return e;
   const int64_t cap = static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1);
   const int grid = static_cast<int>(a.T < cap ? a.T : cap);
-  kern<<<grid, kThreads, smem, st>>>(a, h);
+  kern<<<grid, kThreads, smem, st>>>(a, h, sqrt(static_cast<double>(a.shape.n)));
   count_launch();
   return cudaGetLastError();
+}
+
+template <typename Tin, typename Acc>
+cudaError_t launch_acc(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
+  return a.q != nullptr ? launch_typed<Tin, Acc, true>(a, h, st) : launch_typed<Tin, Acc, false>(a, h, st);
 }
 
 }  // namespace
 
 cudaError_t launch_rotate_generic(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
-  const bool quant = a.q != nullptr;
+  const bool wide = a.shape.n <= 28672;  // fp64 row fits in shared memory
   if (a.dtype == kBF16)
-    return quant ? launch_typed<uint16_t, true>(a, h, st) : launch_typed<uint16_t, false>(a, h, st);
-  return quant ? launch_typed<float, true>(a, h, st) : launch_typed<float, false>(a, h, st);
+    return wide ? launch_acc<uint16_t, double>(a, h, st) : launch_acc<uint16_t, float>(a, h, st);
+  return wide ? launch_acc<float, double>(a, h, st) : launch_acc<float, float>(a, h, st);
 }
 
 }  // namespace signrot

@@ -1,0 +1,767 @@
+// Fused rotate + sign-adjust + asymmetric INT4 quantization on B200 tensor cores (tcgen05 + TMEM).
+//
+// What one token row computes (SignRot abstract and explainer, "The standard fix is rotation" and
+// "SignRot asks one crowd to walk across the hall"): y = diag(s) H diag(D) x / sqrt(n), then the
+// per-token asymmetric 4-bit grid ("Picture the photographer", "Worked example").
+//
+// How it maps onto the hardware. Write the channel index as j = (a, h2, b) with n = 28 * M,
+// a in [0, 28), h2 in [0, 4) (top two bits of the length-M axis) and b in [0, M/4), or for
+// power-of-two n as j = (r, b) with r in [0, 128). The rotation factors as
+//     H = (H_28 kron H_4) kron H_{M/4}      (or H_128 kron H_{n/128})
+// and the first factor is a dense 112 x 112 (128 x 128) block with entries +/-1. It is applied as
+// one tcgen05 MMA chain per token on the exact bf16 inputs (+/-1 times bf16 is exact; fp32
+// accumulation):
+//     A  = rowsign (.) (H_28 kron H_4), 128 x 128 bf16, K-major, SMEM (built once per CTA)
+//     B  = D (.) x viewed as [K = (c, h2) rows][N = b columns], bf16, MN-major, SMEM (TMA tiles)
+//     Dt = A B in TMEM: lane = (h2', a) row, column = b.
+// Each TMEM lane is then one length-M/4 line of the remaining Walsh-Hadamard factor, so every
+// remaining FWHT stage runs inside one thread's registers, and each thread ends up owning a
+// contiguous run of output channels (contiguous packed INT4 stores). The per-token min/max is a
+// warp reduction plus a 4-warp exchange through shared memory.
+//
+// Sign vector from an outlier channel k (signrot_build_sign's form, s_j = sgn(H[j,k] D_k x_k))
+// costs nothing here: with k = (c_k, h2_k, e) the sign factorises into sigma * H_28[a][c_k] *
+// (-1)^popcount(h2 & h2_k) (folded into A's rows) times (-1)^popcount(b & e), which is folded
+// into the FWHT butterflies by swapping the subtraction's operands on the stages whose bit of e
+// is set. A general s vector is applied elementwise in the epilogue instead.
+//
+// Warp roles (320 threads, one CTA per SM, persistent over tokens):
+//   warps 0-3  epilogue: TMEM -> registers, FWHT, min/max, quantize, pack, store (TMEM lane
+//              quadrant = warp index)
+//   warps 4-7  D pass: flip the sign bits of the staged bf16 tile in shared memory
+//   warp 8     TMA producer (one elected lane)
+//   warp 9     TMEM allocator and MMA issuer (one elected lane)
+// Pipeline: TMA -> full[s] -> D pass -> dready[s] -> MMA -> (empty[s], tfull[b]) -> epilogue ->
+// tempty[b] -> MMA. Shared-memory stages form a ring; TMEM holds two token accumulators.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "signrot_device.cuh"
+#include "signrot_internal.h"
+#include "tc_ptx.cuh"
+
+namespace signrot {
+
+// Set (bit 0) by any kernel whose bounded wait gave up; read by signrot_device_error.
+__device__ unsigned int g_device_error = 0;
+
+namespace {
+
+using namespace ptx;
+
+// Eight warps, two per SM sub-partition, so each thread may hold up to 255 registers (each
+// sub-partition has a 16K-register file; a third warp on one would cap every thread at 168).
+constexpr int kThreads = 256;
+constexpr int kEpiWarps = 4;   // warps 0-3
+constexpr int kDWarps = 2;     // warps 4-5
+constexpr int kTmaWarp = 6;
+constexpr int kMmaWarp = 7;
+constexpr uint32_t kABytes = 128 * 128 * 2;  // A: 128 x 128 bf16
+constexpr uint32_t kBoxBytes = 16 * 128;     // one TMA box: 16 rows x 64 bf16 (128 B) = 2 KB
+constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23: fp32 whose ulp is 1
+
+// bit 0: a bounded wait expired; bit 1: the outlier channel index was out of range.
+__device__ __forceinline__ void flag_error(unsigned int bit = 1u) { atomicOr(&g_device_error, bit); }
+
+struct TcParams {
+  int32_t T;
+  int32_t n;
+  int32_t logM;  // F = 28: M = 2^logM; F = 1: unused
+  int32_t stages;
+  const int8_t* d;
+  const int8_t* s;     // general sign vector (kVecSign) or null
+  const int32_t* kp;   // outlier channel (pattern sign) or null
+  const float* xkp;    // its signed calibration value
+  uint8_t* q;
+  float* scale;
+  float* zero;
+  float* y;
+  int64_t ldy;
+  float clip;
+  float inv_sqrt_n;
+  H28Masks h;
+};
+
+// ---------------------------------------------------------------------------- sign bookkeeping
+
+// Structured sign vector: sigma * g(a) * (-1)^popcount(hi & e_hi) * (-1)^popcount(b & e_lo).
+struct SignPlan {
+  float sigma;
+  int32_t c_k;       // F = 28: H_28 column of the outlier (g(a) = H_28[a][c_k])
+  uint32_t e_hi;     // bits of the outlier index that index A's rows (h2 or r)
+  uint32_t e_lo;     // bits that index the TMEM columns: butterfly flips
+  bool active;
+};
+
+template <bool kF28, int kNcol>
+__device__ __forceinline__ SignPlan make_plan(const TcParams& p) {
+  SignPlan sp{1.f, 0, 0u, 0u, false};
+  if (p.kp == nullptr) return sp;
+  const int k = *p.kp;
+  const float xk = *p.xkp;
+  if (k < 0 || k >= p.n) {  // not a channel: report it and apply no sign adjustment
+    flag_error(2u);
+    return sp;
+  }
+  if (xk == 0.f) return sp;  // s_j = sgn(+/-0) = +1 everywhere
+  sp.active = true;
+  sp.sigma = ((xk < 0.f) != (p.d[k] < 0)) ? -1.f : 1.f;
+  constexpr int kLogNcol = kNcol == 64 ? 6 : (kNcol == 128 ? 7 : 8);
+  if (kF28) {
+    const int M = 1 << p.logM;
+    sp.c_k = k >> p.logM;
+    const uint32_t e = static_cast<uint32_t>(k & (M - 1));
+    sp.e_hi = e >> kLogNcol;
+    sp.e_lo = e & (kNcol - 1);
+  } else {
+    sp.e_hi = static_cast<uint32_t>(k) >> kLogNcol;
+    sp.e_lo = static_cast<uint32_t>(k) & (kNcol - 1);
+  }
+  return sp;
+}
+
+// bf16 bit pattern of A[m][k] (m = TMEM lane / output row, k = K index).
+template <bool kF28>
+__device__ __forceinline__ uint16_t a_entry(int m, int k, const SignPlan& sp, const H28Masks& h) {
+  int neg;
+  if (kF28) {
+    const int hp = m >> 5, a = m & 31, c = k >> 2, h2 = k & 3;
+    if (a >= 28 || c >= 28) return 0;
+    neg = static_cast<int>((h.row[a] >> c) & 1u) ^ (__popc(hp & h2) & 1);
+    if (sp.active) neg ^= static_cast<int>((h.row[a] >> sp.c_k) & 1u) ^ (__popc(hp & sp.e_hi) & 1);
+  } else {
+    neg = __popc(m & k) & 1;
+    if (sp.active) neg ^= __popc(m & sp.e_hi) & 1;
+  }
+  if (sp.active && sp.sigma < 0.f) neg ^= 1;
+  return neg ? 0xBF80 : 0x3F80;  // -1 / +1
+}
+
+// K-major 128B-swizzled placement of A[m][k] (8-row x 64-element atoms, K halves 16 KB apart).
+__device__ __forceinline__ uint32_t a_offset(int m, int k) {
+  return static_cast<uint32_t>((k >> 6) * 16384 + (m >> 3) * 1024 + (m & 7) * 128 +
+                               ((((k & 63) >> 3) ^ (m & 7)) << 4) + (k & 7) * 2);
+}
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((addr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(lbo >> 4) << 16) |
+         (static_cast<uint64_t>(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+
+// ---------------------------------------------------------------------------- FWHT in registers
+
+// Butterfly on bit kBit of the column index over pairs p[i] = (w[2i], w[2i+1]).
+template <int kPairs, int kBit, bool kFlip>
+__device__ __forceinline__ void fwht_stage(float2 (&p)[kPairs]) {
+  if constexpr (kBit == 0) {
+#pragma unroll
+    for (int i = 0; i < kPairs; ++i) {
+      const float u = p[i].x, v = p[i].y;
+      p[i].x = u + v;
+      p[i].y = kFlip ? v - u : u - v;
+    }
+  } else {
+    constexpr int hs = 1 << (kBit - 1);
+#pragma unroll
+    for (int i = 0; i < kPairs; ++i) {
+      if ((i & hs) == 0) {
+        const float2 u = p[i], v = p[i + hs];
+        p[i] = __fadd2_rn(u, v);
+        p[i + hs] = kFlip ? fsub2(v, u) : fsub2(u, v);
+      }
+    }
+  }
+}
+
+template <int kPairs, int kBit>
+__device__ __forceinline__ void fwht_stage_rt(float2 (&p)[kPairs], uint32_t flips) {
+  if ((flips >> kBit) & 1u)
+    fwht_stage<kPairs, kBit, true>(p);
+  else
+    fwht_stage<kPairs, kBit, false>(p);
+}
+
+// All stages over kBits bits of the in-thread column index.
+template <int kPairs, int kBits>
+__device__ __forceinline__ void fwht_local(float2 (&p)[kPairs], uint32_t flips) {
+  fwht_stage_rt<kPairs, 0>(p, flips);
+  if (kBits > 1) fwht_stage_rt<kPairs, (kBits > 1 ? 1 : 0)>(p, flips);
+  if (kBits > 2) fwht_stage_rt<kPairs, (kBits > 2 ? 2 : 0)>(p, flips);
+  if (kBits > 3) fwht_stage_rt<kPairs, (kBits > 3 ? 3 : 0)>(p, flips);
+  if (kBits > 4) fwht_stage_rt<kPairs, (kBits > 4 ? 4 : 0)>(p, flips);
+  if (kBits > 5) fwht_stage_rt<kPairs, (kBits > 5 ? 5 : 0)>(p, flips);
+  if (kBits > 6) fwht_stage_rt<kPairs, (kBits > 6 ? 6 : 0)>(p, flips);
+}
+
+// TMEM -> registers: kN pairs (2 * kN consecutive columns from taddr) into p[kOff .. kOff + kN).
+template <int kOff, int kN, int kPairs>
+__device__ __forceinline__ void tmem_load_pairs(uint32_t taddr, float2 (&p)[kPairs]) {
+  static_assert(kN % 16 == 0 && kOff + kN <= kPairs, "whole 32-column loads only");
+#pragma unroll
+  for (int c = 0; c < kN; c += 16) {
+    uint32_t r[32];
+    tmem_ld32(taddr + 2 * c, r);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) p[kOff + c + i] = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+  }
+}
+
+template <int kPairs>
+__device__ __forceinline__ void tmem_store_pairs(uint32_t taddr, const float2 (&p)[kPairs]) {
+#pragma unroll
+  for (int c = 0; c < kPairs; c += 16) {
+    uint32_t r[32];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      r[2 * i] = __float_as_uint(p[c + i].x);
+      r[2 * i + 1] = __float_as_uint(p[c + i].y);
+    }
+    tmem_st32(taddr + 2 * c, r);
+  }
+  tmem_wait_st();
+}
+
+// Elementwise general sign vector: bit r of sbits flips the sign of column r.
+template <int kPairs>
+__device__ __forceinline__ void apply_sign_bits(float2 (&p)[kPairs], const uint32_t* sbits) {
+#pragma unroll
+  for (int i = 0; i < kPairs; ++i) {
+    const int r0 = 2 * i, r1 = 2 * i + 1;
+    const uint32_t m0 = (sbits[r0 >> 5] << (31 - (r0 & 31))) & 0x80000000u;
+    const uint32_t m1 = (sbits[r1 >> 5] << (31 - (r1 & 31))) & 0x80000000u;
+    p[i].x = __uint_as_float(__float_as_uint(p[i].x) ^ m0);
+    p[i].y = __uint_as_float(__float_as_uint(p[i].y) ^ m1);
+  }
+}
+
+template <int kPairs>
+__device__ __forceinline__ void local_minmax(const float2 (&p)[kPairs], float& lo, float& hi) {
+  float l0 = p[0].x, l1 = p[0].y, h0 = p[0].x, h1 = p[0].y;
+#pragma unroll
+  for (int i = 1; i + 1 < kPairs; i += 2) {
+    l0 = fmin3(l0, p[i].x, p[i].y);
+    h0 = fmax3(h0, p[i].x, p[i].y);
+    l1 = fmin3(l1, p[i + 1].x, p[i + 1].y);
+    h1 = fmax3(h1, p[i + 1].x, p[i + 1].y);
+  }
+  if ((kPairs & 1) == 0) {
+    l0 = fmin3(l0, p[kPairs - 1].x, p[kPairs - 1].y);
+    h0 = fmax3(h0, p[kPairs - 1].x, p[kPairs - 1].y);
+  }
+  lo = fminf(lo, fminf(l0, l1));
+  hi = fmaxf(hi, fmaxf(h0, h1));
+}
+
+// Eight consecutive codes -> one u32 of nibbles (element 2i low nibble). u holds the bit
+// patterns of fma(w, c, zero + 1.5*2^23), whose low byte is the code (0..15).
+__device__ __forceinline__ uint32_t pack8(const uint32_t (&u)[8]) {
+  const uint32_t b01 = u[1] * 16u + u[0], b23 = u[3] * 16u + u[2];
+  const uint32_t b45 = u[5] * 16u + u[4], b67 = u[7] * 16u + u[6];
+  const uint32_t w0 = b23 * 256u + b01, w1 = b67 * 256u + b45;
+  return __byte_perm(w0, w1, 0x5410);
+}
+
+// Quantize kPairs pairs (consecutive columns) into packed words (kPairs / 4 of them).
+template <int kPairs, bool kClamp>
+__device__ __forceinline__ void quant_pack(const float2 (&p)[kPairs], float c, float zm, uint32_t* words) {
+  const float2 c2 = make_float2(c, c), z2 = make_float2(zm, zm);
+  const float lo_m = kMagic, hi_m = kMagic + 15.f;
+#pragma unroll
+  for (int g = 0; g < kPairs / 4; ++g) {
+    uint32_t u[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float2 t = __ffma2_rn(p[4 * g + k], c2, z2);
+      if (kClamp) {
+        t.x = fminf(fmaxf(t.x, lo_m), hi_m);
+        t.y = fminf(fmaxf(t.y, lo_m), hi_m);
+      }
+      u[2 * k] = __float_as_uint(t.x);
+      u[2 * k + 1] = __float_as_uint(t.y);
+    }
+    words[g] = pack8(u);
+  }
+}
+
+// Quantize + store one run of 2*kPairs consecutive channels at q_out (16 B aligned).
+template <int kPairs>
+__device__ __forceinline__ void quant_store(const float2 (&p)[kPairs], float c, float zm, bool clamp,
+                                            uint8_t* q_out) {
+  uint32_t words[kPairs / 4];
+  if (clamp)
+    quant_pack<kPairs, true>(p, c, zm, words);
+  else
+    quant_pack<kPairs, false>(p, c, zm, words);
+  uint4* dst = reinterpret_cast<uint4*>(q_out);
+#pragma unroll
+  for (int i = 0; i < kPairs / 16; ++i) dst[i] = make_uint4(words[4 * i], words[4 * i + 1], words[4 * i + 2], words[4 * i + 3]);
+}
+
+template <int kPairs>
+__device__ __forceinline__ void store_y(const float2 (&p)[kPairs], float rs, float* y_out) {
+  float4* dst = reinterpret_cast<float4*>(y_out);
+#pragma unroll
+  for (int i = 0; i < kPairs / 2; ++i)
+    dst[i] = make_float4(p[2 * i].x * rs, p[2 * i].y * rs, p[2 * i + 1].x * rs, p[2 * i + 1].y * rs);
+}
+
+struct TokenGrid {
+  float c;      // w -> y / scale
+  float zm;     // zero + 1.5 * 2^23
+  bool clamp;   // some code of this token falls outside [0, 15] before clamping
+  float scale;
+  float zero;
+};
+
+__device__ __forceinline__ TokenGrid token_grid(float lo_w, float hi_w, float rs, float clip) {
+  const float lo_y = __fmul_rn(lo_w, rs), hi_y = __fmul_rn(hi_w, rs);
+  const QuantGrid g = make_grid(lo_y, hi_y, clip);
+  TokenGrid tg;
+  tg.scale = g.scale;
+  tg.zero = g.zero;
+  tg.c = __fmul_rn(rs, g.inv);
+  tg.zm = __fadd_rn(g.zero, kMagic);
+  // codes are monotone in w, so the row's extremes decide whether any code needs clamping;
+  // a zero-point too large for the 1.5 * 2^23 trick also takes the clamped path
+  const int c_lo = static_cast<int>(__float_as_uint(fmaf(lo_w, tg.c, tg.zm)) - __float_as_uint(kMagic));
+  const int c_hi = static_cast<int>(__float_as_uint(fmaf(hi_w, tg.c, tg.zm)) - __float_as_uint(kMagic));
+  tg.clamp = !(c_lo >= 0 && c_hi <= 15) || fabsf(g.zero) > 4194304.f;
+  return tg;
+}
+
+// ------------------------------------------------------------------------------------- kernel
+
+template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
+__global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcParams p) {
+  constexpr int kKRows = kF28 ? 112 : 128;     // K of the MMA chain
+  constexpr int kKSteps = kKRows / 16;
+  constexpr int kChunksN = kNcol / 64;          // 64-column TMA / swizzle atoms per token
+  constexpr int kBoxesPerChunk = kKRows / 16;
+  constexpr uint32_t kChunkBytes = kKRows * 128;
+  constexpr uint32_t kStageBytes = kChunksN * kChunkBytes;
+  constexpr uint32_t kTmemCols = 2 * kNcol < 32 ? 32 : 2 * kNcol;
+  constexpr int kPairs = kNcol <= 128 ? kNcol / 2 : 64;  // register pairs held per pass
+  constexpr int kStageChunks = kChunksN * kKRows * 8;  // 16-B chunks per stage
+  constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                              (static_cast<uint32_t>(kNcol >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  uint8_t* a_smem = smem;
+  uint32_t* dmask = reinterpret_cast<uint32_t*>(smem + kABytes);  // D sign masks, stage layout
+  uint8_t* ring = smem + kABytes + kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + S * kStageBytes);
+  uint64_t* full = bars;
+  uint64_t* dready = bars + S;
+  uint64_t* empty = bars + 2 * S;
+  uint64_t* tfull = bars + 3 * S;
+  uint64_t* tempty = bars + 3 * S + 2;
+  uint64_t* redbar = bars + 3 * S + 4;  // the 4 epilogue warps' min/max exchange, per TMEM buffer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 6);
+  float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [2 buffers][4 warps][lo, hi]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const SignPlan sp = make_plan<kF28, kNcol>(p);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&dready[i]), kDWarps);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), kEpiWarps);
+      mbar_init(smem_u32(&redbar[i]), kEpiWarps);
+    }
+    fence_mbar_init();
+  }
+  // A = rowsign (.) (H_28 kron H_4) or rowsign (.) H_128, bf16, K-major SW128
+  for (int idx = threadIdx.x; idx < 128 * 128; idx += kThreads) {
+    const int m = idx >> 7, k = idx & 127;
+    *reinterpret_cast<uint16_t*>(a_smem + a_offset(m, k)) = a_entry<kF28>(m, k, sp, p.h);
+  }
+  const int M = kF28 ? (1 << p.logM) : 0;
+  // D as XOR masks on bf16 pairs, in the staged tile's (swizzled) order: 16-B chunk ch holds
+  // row (K index) ch % (kKRows * 8) / 8, logical 8-column segment (slot ^ row) & 7
+  for (int ch = threadIdx.x; ch < kStageChunks; ch += kThreads) {
+    const int nb = ch / (kKRows * 8), rem = ch % (kKRows * 8);
+    const int row = rem >> 3, slot = rem & 7;
+    const int b0 = nb * 64 + ((slot ^ (row & 7)) << 3);
+    const int j0 = kF28 ? (row >> 2) * M + (row & 3) * kNcol + b0 : row * kNcol + b0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      dmask[4 * ch + w] = (p.d[j0 + 2 * w] < 0 ? 0x8000u : 0u) | (p.d[j0 + 2 * w + 1] < 0 ? 0x80000000u : 0u);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmap);
+      int i = 0;
+      for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+        const int st = i % S;
+        if (!mbar_wait(smem_u32(&empty[st]), ((i / S) & 1) ^ 1)) { flag_error(); break; }
+        const uint32_t fb = smem_u32(&full[st]);
+        mbar_arrive_expect_tx(fb, kStageBytes);
+        const uint32_t dst0 = smem_u32(ring + st * kStageBytes);
+#pragma unroll 1
+        for (int nb = 0; nb < kChunksN; ++nb) {
+#pragma unroll 1
+          for (int bx = 0; bx < kBoxesPerChunk; ++bx) {
+            const uint32_t dst = dst0 + nb * kChunkBytes + bx * kBoxBytes;
+            if (kF28)
+              tma_load_4d(dst, &tmap, nb * 64, 0, bx * 4, t, fb);
+            else
+              tma_load_3d(dst, &tmap, nb * 64, bx * 16, t, fb);
+          }
+        }
+      }
+      // do not leave the CTA with copies in flight: wait (bounded) for the last stages issued
+      const int issued = i;
+      for (int j = issued - S > 0 ? issued - S : 0; j < issued; ++j)
+        if (!mbar_wait(smem_u32(&full[j % S]), (j / S) & 1)) { flag_error(); break; }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t a_base = smem_u32(a_smem);
+      int i = 0;
+      for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+        const int st = i % S, tb = i & 1;
+        if (!mbar_wait(smem_u32(&dready[st]), (i / S) & 1)) { flag_error(); break; }
+        if (!mbar_wait(smem_u32(&tempty[tb]), ((i >> 1) & 1) ^ 1)) { flag_error(); break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + tb * kNcol;
+        const uint32_t b_base = smem_u32(ring + st * kStageBytes);
+#pragma unroll
+        for (int ks = 0; ks < kKSteps; ++ks) {
+          const uint64_t ad = smem_desc(a_base + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc(b_base + ks * 2048, kChunkBytes, 1024);
+          mma_bf16(d_tmem, ad, bd, kIdesc, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&empty[st]));
+        mma_commit(smem_u32(&tfull[tb]));
+      }
+      // leave no MMA in flight behind: the last commit must have landed before TMEM is freed
+      if (i > 0 && !mbar_wait(smem_u32(&tfull[(i - 1) & 1]), ((i - 1) >> 1) & 1)) flag_error();
+    }
+  } else if (warp >= kEpiWarps) {
+    // ------------------------------------------------------------------ D pass (warps 4-5)
+    const int td = threadIdx.x - kEpiWarps * 32;
+    const uint4* masks = reinterpret_cast<const uint4*>(dmask);
+    int i = 0;
+    for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+      const int st = i % S;
+      if (!mbar_wait(smem_u32(&full[st]), (i / S) & 1)) { flag_error(); break; }
+      uint4* base = reinterpret_cast<uint4*>(ring + st * kStageBytes);
+#pragma unroll 4
+      for (int ch = td; ch < kStageChunks; ch += kDWarps * 32) {
+        uint4 v = base[ch];
+        const uint4 m = masks[ch];
+        v.x ^= m.x;
+        v.y ^= m.y;
+        v.z ^= m.z;
+        v.w ^= m.w;
+        base[ch] = v;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&dready[st]));
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 0-3)
+    const int quad = warp;
+    const bool active = !kF28 || lane < 28;
+    // this lane's output run: row (h2' = quad, a = lane) or r = quad * 32 + lane
+    const int64_t j0 = kF28 ? static_cast<int64_t>(lane) * M + quad * kNcol : static_cast<int64_t>(quad * 32 + lane) * kNcol;
+    uint32_t sbits[kVecSign ? kNcol / 32 : 1];
+    if (kVecSign) {
+#pragma unroll
+      for (int w = 0; w < kNcol / 32; ++w) {
+        uint32_t b = 0;
+        if (active)
+          for (int r = 0; r < 32; ++r) b |= (p.s[j0 + 32 * w + r] < 0 ? 1u : 0u) << r;
+        sbits[w] = b;
+      }
+    }
+    const uint32_t flips = sp.active ? sp.e_lo : 0u;
+    const float rs = p.inv_sqrt_n;
+    int i = 0;
+    for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+      const int tb = i & 1;
+      if (!mbar_wait(smem_u32(&tfull[tb]), (i >> 1) & 1)) { flag_error(); break; }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tb * kNcol;
+      float2 v[kPairs];
+      float lo = pos_inf(), hi = -pos_inf();
+      if constexpr (kNcol <= 128) {
+        tmem_load_pairs<0, kPairs>(taddr, v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&tempty[tb]));
+        fwht_local<kPairs, (kNcol == 64 ? 6 : 7)>(v, flips);
+        if (kVecSign) apply_sign_bits<kPairs>(v, sbits);
+        if (active) local_minmax<kPairs>(v, lo, hi);
+      } else {
+        // 256 columns: two 128-column halves through the registers, then the top stage
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          tmem_load_pairs<0, kPairs>(taddr + hh * 128, v);
+          fwht_local<kPairs, 7>(v, flips);
+          tmem_store_pairs<kPairs>(taddr + hh * 128, v);
+        }
+        const bool f7 = (flips >> 7) & 1u;
+#pragma unroll 1
+        for (int g = 0; g < 2; ++g) {
+          float2 u[32];
+          tmem_load_pairs<0, 32>(taddr + g * 64, v);
+          tmem_load_pairs<0, 32>(taddr + 128 + g * 64, u);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float2 a = v[k], b = u[k];
+            v[k] = __fadd2_rn(a, b);
+            v[32 + k] = f7 ? fsub2(b, a) : fsub2(a, b);
+          }
+          if (kVecSign) {
+            const uint32_t sb[2] = {sbits[2 * g], sbits[2 * g + 1]};
+            const uint32_t sb2[2] = {sbits[4 + 2 * g], sbits[4 + 2 * g + 1]};
+            float2 lo_half[32], hi_half[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) { lo_half[k] = v[k]; hi_half[k] = v[32 + k]; }
+            apply_sign_bits<32>(lo_half, sb);
+            apply_sign_bits<32>(hi_half, sb2);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) { v[k] = lo_half[k]; v[32 + k] = hi_half[k]; }
+          }
+          if (active) local_minmax<64>(v, lo, hi);
+        }
+      }
+      // token min/max: warp, then the 4 epilogue warps through shared memory
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      }
+      if (lane == 0) {
+        red[(tb * 4 + quad) * 2] = lo;
+        red[(tb * 4 + quad) * 2 + 1] = hi;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&redbar[tb]));
+      if (!mbar_wait(smem_u32(&redbar[tb]), (i >> 1) & 1)) { flag_error(); break; }
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        lo = fminf(lo, red[(tb * 4 + w) * 2]);
+        hi = fmaxf(hi, red[(tb * 4 + w) * 2 + 1]);
+      }
+      if (kQuant) {
+        const TokenGrid g = token_grid(lo, hi, rs, p.clip);
+        if (threadIdx.x == 0) {
+          p.scale[t] = g.scale;
+          p.zero[t] = g.zero;
+        }
+        uint8_t* qrow = p.q + static_cast<int64_t>(t) * (p.n >> 1);
+        if constexpr (kNcol <= 128) {
+          if (active) quant_store<kPairs>(v, g.c, g.zm, g.clamp, qrow + (j0 >> 1));
+        } else {
+          const bool f7 = (flips >> 7) & 1u;
+#pragma unroll 1
+          for (int gg = 0; gg < 2; ++gg) {
+            float2 u[32], lo_half[32], hi_half[32];
+            tmem_load_pairs<0, 32>(taddr + gg * 64, lo_half);
+            tmem_load_pairs<0, 32>(taddr + 128 + gg * 64, u);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const float2 a = lo_half[k], b = u[k];
+              lo_half[k] = __fadd2_rn(a, b);
+              hi_half[k] = f7 ? fsub2(b, a) : fsub2(a, b);
+            }
+            if (kVecSign) {
+              const uint32_t sb[2] = {sbits[2 * gg], sbits[2 * gg + 1]};
+              const uint32_t sb2[2] = {sbits[4 + 2 * gg], sbits[4 + 2 * gg + 1]};
+              apply_sign_bits<32>(lo_half, sb);
+              apply_sign_bits<32>(hi_half, sb2);
+            }
+            if (active) {
+              quant_store<32>(lo_half, g.c, g.zm, g.clamp, qrow + ((j0 + gg * 64) >> 1));
+              quant_store<32>(hi_half, g.c, g.zm, g.clamp, qrow + ((j0 + 128 + gg * 64) >> 1));
+            }
+          }
+        }
+      } else {
+        float* yrow = p.y + static_cast<int64_t>(t) * p.ldy;
+        if constexpr (kNcol <= 128) {
+          if (active) store_y<kPairs>(v, rs, yrow + j0);
+        } else {
+          const bool f7 = (flips >> 7) & 1u;
+#pragma unroll 1
+          for (int gg = 0; gg < 2; ++gg) {
+            float2 u[32], lo_half[32], hi_half[32];
+            tmem_load_pairs<0, 32>(taddr + gg * 64, lo_half);
+            tmem_load_pairs<0, 32>(taddr + 128 + gg * 64, u);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const float2 a = lo_half[k], b = u[k];
+              lo_half[k] = __fadd2_rn(a, b);
+              hi_half[k] = f7 ? fsub2(b, a) : fsub2(a, b);
+            }
+            if (kVecSign) {
+              const uint32_t sb[2] = {sbits[2 * gg], sbits[2 * gg + 1]};
+              const uint32_t sb2[2] = {sbits[4 + 2 * gg], sbits[4 + 2 * gg + 1]};
+              apply_sign_bits<32>(lo_half, sb);
+              apply_sign_bits<32>(hi_half, sb2);
+            }
+            if (active) {
+              store_y<32>(lo_half, rs, yrow + j0 + gg * 64);
+              store_y<32>(hi_half, rs, yrow + j0 + 128 + gg * 64);
+            }
+          }
+        }
+      }
+      if constexpr (kNcol > 128) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&tempty[tb]));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------- host
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
+cudaError_t launch_tc(const CUtensorMap& tmap, const TcParams& p0, cudaStream_t st) {
+  constexpr int kKRows = kF28 ? 112 : 128;
+  constexpr uint32_t kStageBytes = (kNcol / 64) * kKRows * 128;
+  constexpr uint32_t kSmemBudget = 227 * 1024 - 1024 - kABytes - kStageBytes - 512;
+  TcParams p = p0;
+  p.stages = static_cast<int>(kSmemBudget / kStageBytes);
+  if (p.stages > 8) p.stages = 8;
+  const size_t smem = 1024 + kABytes + kStageBytes + static_cast<size_t>(p.stages) * kStageBytes + 512;
+  auto kern = rotq_tc_kernel<kNcol, kF28, kVecSign, kQuant>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = p.T < sms ? p.T : sms;
+  kern<<<grid, kThreads, smem, st>>>(tmap, p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <int kNcol, bool kF28>
+cudaError_t dispatch_mode(const CUtensorMap& tmap, const TcParams& p, bool vec_sign, bool quant, cudaStream_t st) {
+  if (vec_sign)
+    return quant ? launch_tc<kNcol, kF28, true, true>(tmap, p, st) : launch_tc<kNcol, kF28, true, false>(tmap, p, st);
+  return quant ? launch_tc<kNcol, kF28, false, true>(tmap, p, st) : launch_tc<kNcol, kF28, false, false>(tmap, p, st);
+}
+
+}  // namespace
+
+cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
+  if (a.dtype != kBF16 || a.T <= 0 || a.T > 0x7fffffff) return cudaErrorNotSupported;
+  const bool f28 = a.shape.F == 28;
+  const int ncol = f28 ? (1 << a.shape.logM) / 4 : a.shape.n / 128;
+  if (ncol != 64 && ncol != 128 && ncol != 256) return cudaErrorNotSupported;
+  if (reinterpret_cast<uintptr_t>(a.x) % 16 != 0 || a.ld % 8 != 0) return cudaErrorNotSupported;
+  const bool quant = a.q != nullptr;
+  if (quant && reinterpret_cast<uintptr_t>(a.q) % 16 != 0) return cudaErrorNotSupported;
+  if (!quant && (reinterpret_cast<uintptr_t>(a.y) % 16 != 0 || a.ldy % 4 != 0)) return cudaErrorNotSupported;
+  auto encode = encode_fn();
+  if (encode == nullptr) return cudaErrorNotSupported;
+
+  CUtensorMap tmap;
+  CUresult r;
+  const cuuint32_t elem_strides[4] = {1, 1, 1, 1};
+  if (f28) {
+    const int M = 1 << a.shape.logM;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(ncol), 4, 28, static_cast<cuuint64_t>(a.T)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(ncol) * 2, static_cast<cuuint64_t>(M) * 2,
+                                   static_cast<cuuint64_t>(a.ld) * 2};
+    const cuuint32_t box[4] = {64, 4, 4, 1};
+    r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(a.x), dims, strides, box, elem_strides,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(ncol), 128, static_cast<cuuint64_t>(a.T)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ncol) * 2, static_cast<cuuint64_t>(a.ld) * 2};
+    const cuuint32_t box[3] = {64, 16, 1};
+    r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.x), dims, strides, box, elem_strides,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  if (r != CUDA_SUCCESS) return cudaErrorNotSupported;
+
+  TcParams p{};
+  p.T = static_cast<int32_t>(a.T);
+  p.n = a.shape.n;
+  p.logM = a.shape.logM;
+  p.d = a.d;
+  p.s = a.s;
+  p.kp = a.kp;
+  p.xkp = a.xkp;
+  p.q = a.q;
+  p.scale = a.scale;
+  p.zero = a.zero;
+  p.y = a.y;
+  p.ldy = a.ldy;
+  p.clip = a.clip;
+  p.inv_sqrt_n = a.inv_sqrt_n;
+  p.h = h;
+  const bool vec = a.s != nullptr && a.kp == nullptr;
+  if (f28) {
+    if (ncol == 64) return dispatch_mode<64, true>(tmap, p, vec, quant, st);
+    if (ncol == 128) return dispatch_mode<128, true>(tmap, p, vec, quant, st);
+    return dispatch_mode<256, true>(tmap, p, vec, quant, st);
+  }
+  if (ncol == 64) return dispatch_mode<64, false>(tmap, p, vec, quant, st);
+  if (ncol == 128) return dispatch_mode<128, false>(tmap, p, vec, quant, st);
+  return dispatch_mode<256, false>(tmap, p, vec, quant, st);
+}
+
+cudaError_t read_device_error(uint32_t* out, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_device_error, sizeof(uint32_t));
+  if (e != cudaSuccess || !clear) return e;
+  const uint32_t zero = 0;
+  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(uint32_t));
+}
+
+}  // namespace signrot

@@ -77,6 +77,35 @@ const H28State& h28_state() {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Two copy/compute streams and their join events per device, created on first use and kept for
+// the life of the process (the host-buffer entry point allocates nothing per call).
+struct HostStreams {
+  cudaStream_t s[2];
+  cudaEvent_t start;
+  cudaEvent_t done[2];
+};
+
+HostStreams* host_streams(int dev) {
+  static std::mutex mu;
+  static HostStreams* per_dev[64] = {};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> guard(mu);
+  if (per_dev[dev] == nullptr) {
+    auto* h = new HostStreams{};
+    bool ok = cudaStreamCreateWithFlags(&h->s[0], cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&h->s[1], cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->start, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->done[0], cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->done[1], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      delete h;
+      return nullptr;
+    }
+    per_dev[dev] = h;
+  }
+  return per_dev[dev];
+}
+
 signrot_status check_rows(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
                           signrot::Shape* sh) {
   if (dtype != SIGNROT_BF16 && dtype != SIGNROT_F32)
@@ -101,6 +130,69 @@ signrot_status run_rotate(signrot::RotateArgs& a, cudaStream_t st) {
   }
   if (e != cudaSuccess) return cuda_fail(e, "rotate launch");
   return SIGNROT_OK;
+}
+
+signrot_status rotate_impl(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                           const int8_t* d, const int8_t* s, const int32_t* kp, const float* xkp,
+                           float* y, int64_t ldy, void* stream) {
+  g_last_error[0] = '\0';
+  signrot::Shape sh;
+  signrot_status st = check_rows(x, dtype, T, n, ld, &sh);
+  if (st != SIGNROT_OK) return st;
+  if (d == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "d is NULL");
+  if (T > 0 && y == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < n) return fail(SIGNROT_ERR_INVALID_ARG, "ldy < n");
+  if (!aligned(y, 4)) return fail(SIGNROT_ERR_ALIGNMENT, "y is not 4-byte aligned");
+  if (!aligned(kp, 4) || !aligned(xkp, 4)) return fail(SIGNROT_ERR_ALIGNMENT, "k or xk misaligned");
+  if (T == 0) return SIGNROT_OK;
+  signrot::RotateArgs a{};
+  a.x = x;
+  a.dtype = dtype;
+  a.T = T;
+  a.ld = ld;
+  a.shape = sh;
+  a.d = d;
+  a.s = s;
+  a.kp = kp;
+  a.xkp = xkp;
+  a.y = y;
+  a.ldy = ldy;
+  a.clip = 1.f;
+  return run_rotate(a, static_cast<cudaStream_t>(stream));
+}
+
+signrot_status rotate_quant_impl(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                 const int8_t* d, const int8_t* s, const int32_t* kp, const float* xkp,
+                                 int32_t bits, float clip, uint8_t* q, float* scale, float* zero,
+                                 void* stream) {
+  g_last_error[0] = '\0';
+  signrot::Shape sh;
+  signrot_status st = check_rows(x, dtype, T, n, ld, &sh);
+  if (st != SIGNROT_OK) return st;
+  if (bits != 4) return fail(SIGNROT_ERR_UNSUPPORTED, "bits = %d; only 4 is supported", bits);
+  if (!(clip > 0.f && clip <= 1.f)) return fail(SIGNROT_ERR_UNSUPPORTED, "clip must lie in (0, 1]");
+  if (d == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "d is NULL");
+  if (T > 0 && (q == nullptr || scale == nullptr || zero == nullptr))
+    return fail(SIGNROT_ERR_INVALID_ARG, "q, scale and zero must be device pointers");
+  if (!aligned(scale, 4) || !aligned(zero, 4))
+    return fail(SIGNROT_ERR_ALIGNMENT, "scale / zero not 4-byte aligned");
+  if (!aligned(kp, 4) || !aligned(xkp, 4)) return fail(SIGNROT_ERR_ALIGNMENT, "k or xk misaligned");
+  if (T == 0) return SIGNROT_OK;
+  signrot::RotateArgs a{};
+  a.x = x;
+  a.dtype = dtype;
+  a.T = T;
+  a.ld = ld;
+  a.shape = sh;
+  a.d = d;
+  a.s = s;
+  a.kp = kp;
+  a.xkp = xkp;
+  a.q = q;
+  a.scale = scale;
+  a.zero = zero;
+  a.clip = clip;
+  return run_rotate(a, static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -151,57 +243,126 @@ signrot_status signrot_build_sign(int32_t n, const int32_t* k, const float* xk, 
 signrot_status signrot_rotate(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
                               const int8_t* d, const int8_t* s, float* y, int64_t ldy,
                               void* stream) {
-  g_last_error[0] = '\0';
-  signrot::Shape sh;
-  signrot_status st = check_rows(x, dtype, T, n, ld, &sh);
-  if (st != SIGNROT_OK) return st;
-  if (d == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "d is NULL");
-  if (T > 0 && y == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "y is NULL");
-  if (ldy < n) return fail(SIGNROT_ERR_INVALID_ARG, "ldy < n");
-  if (!aligned(y, 4)) return fail(SIGNROT_ERR_ALIGNMENT, "y is not 4-byte aligned");
-  if (T == 0) return SIGNROT_OK;
-  signrot::RotateArgs a{};
-  a.x = x;
-  a.dtype = dtype;
-  a.T = T;
-  a.ld = ld;
-  a.shape = sh;
-  a.d = d;
-  a.s = s;
-  a.y = y;
-  a.ldy = ldy;
-  a.clip = 1.f;
-  return run_rotate(a, static_cast<cudaStream_t>(stream));
+  return rotate_impl(x, dtype, T, n, ld, d, s, nullptr, nullptr, y, ldy, stream);
+}
+
+signrot_status signrot_rotate_outlier(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                      const int8_t* d, const int32_t* k, const float* xk, float* y,
+                                      int64_t ldy, void* stream) {
+  if (k == nullptr || xk == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "k and xk must be device pointers");
+  return rotate_impl(x, dtype, T, n, ld, d, nullptr, k, xk, y, ldy, stream);
 }
 
 signrot_status signrot_rotate_quant(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
                                     const int8_t* d, const int8_t* s, int32_t bits, float clip,
                                     uint8_t* q, float* scale, float* zero, void* stream) {
+  return rotate_quant_impl(x, dtype, T, n, ld, d, s, nullptr, nullptr, bits, clip, q, scale, zero, stream);
+}
+
+signrot_status signrot_rotate_quant_outlier(const void* x, int32_t dtype, int64_t T, int32_t n,
+                                            int64_t ld, const int8_t* d, const int32_t* k,
+                                            const float* xk, int32_t bits, float clip, uint8_t* q,
+                                            float* scale, float* zero, void* stream) {
+  if (k == nullptr || xk == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "k and xk must be device pointers");
+  return rotate_quant_impl(x, dtype, T, n, ld, d, nullptr, k, xk, bits, clip, q, scale, zero, stream);
+}
+
+size_t signrot_host_bytes_per_token(int32_t n, int32_t dtype) {
+  if (n <= 0) return 0;
+  const size_t in_row = static_cast<size_t>(n) * (dtype == SIGNROT_F32 ? 4 : 2);
+  return in_row + static_cast<size_t>(n) / 2 + 8;
+}
+
+signrot_status signrot_rotate_quant_host(const void* x_host, int32_t dtype, int64_t T, int32_t n,
+                                         int64_t ld, const int8_t* d, const int8_t* s,
+                                         const int32_t* k, const float* xk, int32_t bits, float clip,
+                                         uint8_t* q_host, float* scale_host, float* zero_host,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
   g_last_error[0] = '\0';
   signrot::Shape sh;
-  signrot_status st = check_rows(x, dtype, T, n, ld, &sh);
+  signrot_status st = check_rows(x_host, dtype, T, n, ld, &sh);
   if (st != SIGNROT_OK) return st;
   if (bits != 4) return fail(SIGNROT_ERR_UNSUPPORTED, "bits = %d; only 4 is supported", bits);
   if (!(clip > 0.f && clip <= 1.f)) return fail(SIGNROT_ERR_UNSUPPORTED, "clip must lie in (0, 1]");
   if (d == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "d is NULL");
-  if (T > 0 && (q == nullptr || scale == nullptr || zero == nullptr))
-    return fail(SIGNROT_ERR_INVALID_ARG, "q, scale and zero must be device pointers");
-  if (!aligned(scale, 4) || !aligned(zero, 4))
-    return fail(SIGNROT_ERR_ALIGNMENT, "scale / zero not 4-byte aligned");
+  if ((k == nullptr) != (xk == nullptr)) return fail(SIGNROT_ERR_INVALID_ARG, "give both k and xk, or neither");
+  if (k != nullptr && s != nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "s and (k, xk) are exclusive");
+  if (T > 0 && (q_host == nullptr || scale_host == nullptr || zero_host == nullptr || workspace == nullptr))
+    return fail(SIGNROT_ERR_INVALID_ARG, "q_host, scale_host, zero_host and workspace are required");
+  if (!aligned(workspace, 16)) return fail(SIGNROT_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
   if (T == 0) return SIGNROT_OK;
-  signrot::RotateArgs a{};
-  a.x = x;
-  a.dtype = dtype;
-  a.T = T;
-  a.ld = ld;
-  a.shape = sh;
-  a.d = d;
-  a.s = s;
-  a.q = q;
-  a.scale = scale;
-  a.zero = zero;
-  a.clip = clip;
-  return run_rotate(a, static_cast<cudaStream_t>(stream));
+  const size_t esz = dtype == SIGNROT_F32 ? 4 : 2;
+  const size_t in_row = static_cast<size_t>(n) * esz, q_row = static_cast<size_t>(n) / 2;
+  const size_t per_token = signrot_host_bytes_per_token(n, dtype);
+  const size_t slack = 64;  // 16-byte alignment of the three buffers in a slot
+  if (workspace_bytes < 2 * (per_token + slack))
+    return fail(SIGNROT_ERR_INVALID_ARG, "workspace of %zu bytes holds no token (need >= %zu)", workspace_bytes,
+                2 * (per_token + slack));
+  const int64_t chunk_cap = static_cast<int64_t>((workspace_bytes / 2 - slack) / per_token);
+  const int64_t chunk = chunk_cap < T ? chunk_cap : T;
+  const auto up16 = [](size_t v) { return (v + 15) & ~size_t(15); };
+  const size_t off_q = up16(static_cast<size_t>(chunk) * in_row);
+  const size_t off_s = up16(off_q + static_cast<size_t>(chunk) * q_row);
+  const size_t off_z = up16(off_s + static_cast<size_t>(chunk) * 4);
+  const size_t slot_bytes = up16(off_z + static_cast<size_t>(chunk) * 4);
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  HostStreams* hs = host_streams(dev);
+  if (hs == nullptr) return fail(SIGNROT_ERR_CUDA, "could not create the copy streams");
+  auto caller = static_cast<cudaStream_t>(stream);
+  if ((e = cudaEventRecord(hs->start, caller)) != cudaSuccess) return cuda_fail(e, "event record");
+  for (int i = 0; i < 2; ++i)
+    if ((e = cudaStreamWaitEvent(hs->s[i], hs->start, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+
+  const auto* xb = static_cast<const uint8_t*>(x_host);
+  auto* ws = static_cast<uint8_t*>(workspace);
+  for (int64_t t0 = 0, c = 0; t0 < T; t0 += chunk, ++c) {
+    const int64_t tc = T - t0 < chunk ? T - t0 : chunk;
+    cudaStream_t cs = hs->s[c & 1];
+    uint8_t* slot = ws + (c & 1) * slot_bytes;
+    e = cudaMemcpy2DAsync(slot, in_row, xb + static_cast<size_t>(t0) * ld * esz, static_cast<size_t>(ld) * esz, in_row,
+                          static_cast<size_t>(tc), cudaMemcpyHostToDevice, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "rows to device");
+    signrot::RotateArgs a{};
+    a.x = slot;
+    a.dtype = dtype;
+    a.T = tc;
+    a.ld = n;
+    a.shape = sh;
+    a.d = d;
+    a.s = s;
+    a.kp = k;
+    a.xkp = xk;
+    a.q = slot + off_q;
+    a.scale = reinterpret_cast<float*>(slot + off_s);
+    a.zero = reinterpret_cast<float*>(slot + off_z);
+    a.clip = clip;
+    if ((st = run_rotate(a, cs)) != SIGNROT_OK) return st;
+    if ((e = cudaMemcpyAsync(q_host + static_cast<size_t>(t0) * q_row, a.q, static_cast<size_t>(tc) * q_row,
+                             cudaMemcpyDeviceToHost, cs)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(scale_host + t0, a.scale, static_cast<size_t>(tc) * 4, cudaMemcpyDeviceToHost, cs)) !=
+            cudaSuccess ||
+        (e = cudaMemcpyAsync(zero_host + t0, a.zero, static_cast<size_t>(tc) * 4, cudaMemcpyDeviceToHost, cs)) !=
+            cudaSuccess)
+      return cuda_fail(e, "codes to host");
+  }
+  for (int i = 0; i < 2; ++i) {
+    if ((e = cudaEventRecord(hs->done[i], hs->s[i])) != cudaSuccess) return cuda_fail(e, "event record");
+    if ((e = cudaStreamWaitEvent(caller, hs->done[i], 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+  }
+  return SIGNROT_OK;
+}
+
+signrot_status signrot_device_error(int32_t* code, int32_t clear) {
+  g_last_error[0] = '\0';
+  if (code == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "code is NULL");
+  uint32_t v = 0;
+  cudaError_t e = signrot::read_device_error(&v, clear != 0);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  *code = static_cast<int32_t>(v);
+  return SIGNROT_OK;
 }
 
 signrot_status signrot_get_h28(int8_t* out) {

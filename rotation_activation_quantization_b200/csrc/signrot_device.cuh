@@ -67,6 +67,12 @@ __device__ __forceinline__ QuantGrid make_grid(float lo, float hi, float clip) {
   return g;
 }
 
+// code = clamp(rne(y / scale) + zero, 0, 15) with a true IEEE division (the formula as written).
+__device__ __forceinline__ uint32_t quant_code_div(float y, const QuantGrid& g) {
+  const float v = __fadd_rn(rintf(__fdiv_rn(y, g.scale)), g.zero);
+  return static_cast<uint32_t>(fminf(fmaxf(v, 0.f), 15.f));
+}
+
 // code = clamp(rne(y / scale) + zero, 0, 15), with y / scale taken as y * fp32(1/scale).
 __device__ __forceinline__ uint32_t quant_code(float y, const QuantGrid& g) {
   const float v = __fadd_rn(rintf(__fmul_rn(y, g.inv)), g.zero);

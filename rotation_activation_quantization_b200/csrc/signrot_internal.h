@@ -36,6 +36,9 @@ struct RotateArgs {
   Shape shape;
   const int8_t* d;  // [n] +/-1
   const int8_t* s;  // [n] +/-1 or null
+  // sign vector given by its outlier channel instead (s_j = sgn(H[j,k] D_k x_k)), read on device
+  const int32_t* kp;
+  const float* xkp;
   // check path (fp32 y) -- y != null
   float* y;
   int64_t ldy;
@@ -53,6 +56,9 @@ cudaError_t launch_rotate_generic(const RotateArgs& a, const H28Masks& h, cudaSt
 // Fast fused kernels for the shapes they cover; return cudaErrorNotSupported when the shape or
 // the alignment is not theirs (the caller then uses the generic kernel).
 cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStream_t st);
+
+// Reads (and optionally clears) the device error word set by a kernel whose bounded wait expired.
+cudaError_t read_device_error(uint32_t* out, bool clear);
 
 struct CalibArgs {
   const void* x;

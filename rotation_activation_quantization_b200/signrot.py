@@ -27,6 +27,13 @@ _SIGNATURES = {
     "signrot_rotate": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_i64, _c_p],
     "signrot_rotate_quant": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_i32, _c_f,
                              _c_p, _c_p, _c_p, _c_p],
+    "signrot_rotate_outlier": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_p],
+    "signrot_rotate_quant_outlier": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_i32, _c_f,
+                                     _c_p, _c_p, _c_p, _c_p],
+    "signrot_device_error": [_c_p, _c_i32],
+    "signrot_rotate_quant_host": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_f,
+                                  _c_p, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p],
+    "signrot_host_bytes_per_token": [_c_i32, _c_i32],
     "signrot_get_h28": [_c_p],
     "signrot_supported_n": [_c_i32],
     "signrot_status_string": [_c_i32],
@@ -62,6 +69,7 @@ def lib() -> ctypes.CDLL:
         L.signrot_status_string.restype = ctypes.c_char_p
         L.signrot_last_error.restype = ctypes.c_char_p
         L.signrot_kernel_launches.restype = ctypes.c_uint64
+        L.signrot_host_bytes_per_token.restype = ctypes.c_size_t
         _lib = L
     return _lib
 
@@ -188,4 +196,81 @@ def rotate_quant(x: torch.Tensor, d: torch.Tensor, s: torch.Tensor | None = None
         st = lib().signrot_rotate_quant(_ptr(x), _dtype_code(x), T, n, ld, _ptr(d), _ptr(s), int(bits),
                                         float(clip), _ptr(q), _ptr(scale), _ptr(zero), _stream(dev, stream))
     _check("signrot_rotate_quant", st)
+    return q, scale, zero
+
+
+def rotate_outlier(x: torch.Tensor, d: torch.Tensor, k: torch.Tensor, xk: torch.Tensor,
+                   out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """fp32 rotation with the sign vector given by its outlier channel (k, x_k on the device)."""
+    T, n, ld = _rows(x)
+    dev = x.device
+    _need(d, dev, torch.int8, n, "d")
+    _need(k, dev, torch.int32, 1, "k")
+    _need(xk, dev, torch.float32, 1, "xk")
+    out = torch.empty((T, n), dtype=torch.float32, device=dev) if out is None else out
+    if out.shape != (T, n) or out.stride(1) != 1 or out.dtype != torch.float32 or out.device != dev:
+        raise ValueError("out must be a float32 [T, n] tensor with unit stride along n on x's device")
+    ldy = out.stride(0) if T > 1 else n
+    with torch.cuda.device(dev):
+        st = lib().signrot_rotate_outlier(_ptr(x), _dtype_code(x), T, n, ld, _ptr(d), _ptr(k), _ptr(xk),
+                                          _ptr(out), ldy, _stream(dev, stream))
+    _check("signrot_rotate_outlier", st)
+    return out
+
+
+def rotate_quant_outlier(x: torch.Tensor, d: torch.Tensor, k: torch.Tensor, xk: torch.Tensor, bits: int = 4,
+                         clip: float = 1.0, q: torch.Tensor | None = None, scale: torch.Tensor | None = None,
+                         zero: torch.Tensor | None = None, stream=None):
+    """The fused path with the sign vector folded in from (k, x_k): (q, scale, zero)."""
+    T, n, ld = _rows(x)
+    dev = x.device
+    _need(d, dev, torch.int8, n, "d")
+    _need(k, dev, torch.int32, 1, "k")
+    _need(xk, dev, torch.float32, 1, "xk")
+    q = torch.empty((T, n // 2), dtype=torch.uint8, device=dev) if q is None else q
+    scale = torch.empty(T, dtype=torch.float32, device=dev) if scale is None else scale
+    zero = torch.empty(T, dtype=torch.float32, device=dev) if zero is None else zero
+    _need(q, dev, torch.uint8, T * (n // 2), "q")
+    _need(scale, dev, torch.float32, T, "scale")
+    _need(zero, dev, torch.float32, T, "zero")
+    with torch.cuda.device(dev):
+        st = lib().signrot_rotate_quant_outlier(_ptr(x), _dtype_code(x), T, n, ld, _ptr(d), _ptr(k), _ptr(xk),
+                                                int(bits), float(clip), _ptr(q), _ptr(scale), _ptr(zero),
+                                                _stream(dev, stream))
+    _check("signrot_rotate_quant_outlier", st)
+    return q, scale, zero
+
+
+def device_error(clear: bool = True) -> int:
+    """The current device's error word (0 = none); synchronous."""
+    code = ctypes.c_int32(0)
+    _check("signrot_device_error", lib().signrot_device_error(ctypes.byref(code), int(bool(clear))))
+    return int(code.value)
+
+
+def host_bytes_per_token(n: int, dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(lib().signrot_host_bytes_per_token(int(n), BF16 if dtype == torch.bfloat16 else F32))
+
+
+def rotate_quant_host(x: torch.Tensor, d: torch.Tensor, q: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
+                      workspace: torch.Tensor, s: torch.Tensor | None = None, k: torch.Tensor | None = None,
+                      xk: torch.Tensor | None = None, bits: int = 4, clip: float = 1.0, device=None, stream=None):
+    """The fused path between host buffers (x, q, scale, zero on the CPU, pinned for overlap),
+    streamed through a device workspace. Enqueued on the current stream of ``device``."""
+    if x.dim() != 2 or x.stride(1) != 1 or x.is_cuda:
+        raise ValueError("x must be a 2-D host tensor with unit stride along n")
+    T, n = x.shape
+    ld = x.stride(0) if T > 1 else n
+    dev = torch.device(device) if device is not None else d.device
+    if not workspace.is_cuda or workspace.device != dev:
+        raise ValueError("workspace must be a device tensor on the same device as d")
+    for t, name in ((q, "q"), (scale, "scale"), (zero, "zero")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor")
+    with torch.cuda.device(dev):
+        st = lib().signrot_rotate_quant_host(
+            _ptr(x), _dtype_code(x), T, n, ld, _ptr(d), _ptr(s), _ptr(k), _ptr(xk), int(bits), float(clip),
+            _ptr(q), _ptr(scale), _ptr(zero), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(dev, stream))
+    _check("signrot_rotate_quant_host", st)
     return q, scale, zero

@@ -11,10 +11,21 @@ Tolerances (the SignRot build's stated acceptance bar):
 
 A token whose zero-point took the other side of a tie is compared against the oracle's codes
 recomputed with that zero (both are correct roundings of the same tie).
+
+Conditioning. The quantizer's inputs are differences of fp32 values: hi - lo, and y / scale with
+|y| / scale up to |zero|. Where a row's spread is tiny next to its magnitude (a massive outlier on
+a very short row, e.g. n = 2), fp32 rounding of y alone moves scale and zero by more than the bar
+above. ``strict=False`` widens each token's windows by a bound on that rounding:
+    delta_t = (log2(M) + F - 1 + 2) * 2^-24 * ||x_t||_1 / sqrt(n)
+(each output is a sum with at most log2(M) + F - 1 additions on any path, every partial sum is
+bounded by ||x_t||_1, plus the 1/sqrt(n) product and the sign flip), and requires of every code
+that it dequantizes to within half a step (+ delta_t) of the exact rotation.
 """
 from __future__ import annotations
 
+import json
 import math
+import os
 
 import numpy as np
 
@@ -25,10 +36,19 @@ ROT_MAX_ABS = 1e-2
 SCALE_REL = 1e-5
 TIE_EPS = 1e-3
 TIE_FRAC = 1e-4
+U32 = 2.0 ** -24
 
 
 def _half_dist(v: np.ndarray) -> np.ndarray:
     return np.abs(v - np.floor(v) - 0.5)
+
+
+def fp32_rotation_bound(x64: np.ndarray) -> np.ndarray:
+    """Per-token bound on |y_fp32 - y_exact| for the rotation computed in fp32."""
+    T, n = x64.shape
+    F, M = o.factor_n(n)
+    S = int(round(math.log2(M))) + (F - 1) + 2
+    return S * U32 * np.abs(x64).sum(axis=1) / math.sqrt(n)
 
 
 def check_rotation(y_gpu: np.ndarray, y_ref: np.ndarray) -> dict:
@@ -43,36 +63,78 @@ def check_rotation(y_gpu: np.ndarray, y_ref: np.ndarray) -> dict:
 
 
 def check_quant(q_gpu: np.ndarray, scale_gpu: np.ndarray, zero_gpu: np.ndarray, y_ref: np.ndarray,
-                clip: float = 1.0) -> dict:
+                clip: float = 1.0, x64: np.ndarray | None = None, strict: bool = True) -> dict:
     T, n = y_ref.shape
     codes_ref, scale_ref, zero_ref = o.quantize_asym(y_ref, clip=clip)
     vpre, zpre = o.asym_preround(y_ref, clip=clip)
     codes_gpu = o.unpack_nibbles(np.asarray(q_gpu, dtype=np.uint8).reshape(T, n // 2))
     scale_gpu = np.asarray(scale_gpu, dtype=np.float32)
     zero_gpu = np.asarray(zero_gpu, dtype=np.float32)
+    y32 = y_ref.astype(np.float32)
+    lo_c = y32.min(axis=1).astype(np.float64) * clip
+    hi_c = y32.max(axis=1).astype(np.float64) * clip
+    rng = np.maximum(hi_c - lo_c, 1e-30)
+
+    if strict:
+        delta = np.zeros(T)
+    else:
+        assert x64 is not None, "strict=False needs the input rows"
+        delta = fp32_rotation_bound(x64) + np.abs(y_ref).max(axis=1) * U32
+    srel_tol = SCALE_REL + 2.0 * clip * delta / rng
+    amax = np.abs(y_ref).max(axis=1)
+    if strict:  # the stated bar as is: windows of TIE_EPS, every element counts toward TIE_FRAC
+        w_code = np.full(T, TIE_EPS)
+        w_zero = np.full(T, TIE_EPS)
+    else:
+        w_code = np.maximum(TIE_EPS, delta / scale_ref + (amax / scale_ref) * srel_tol * (1 + 1e-3))
+        w_zero = np.maximum(TIE_EPS, clip * delta / scale_ref + (np.abs(lo_c) / scale_ref) * srel_tol * (1 + 1e-3))
 
     srel = np.abs(scale_gpu.astype(np.float64) - scale_ref) / np.abs(scale_ref)
-    assert (srel <= SCALE_REL).all(), f"scale rel err {srel.max():.3e} > {SCALE_REL}"
+    assert (srel <= srel_tol).all(), f"scale rel err {srel.max():.3e} > {srel_tol[np.argmax(srel)]:.3e}"
 
     zdiff = zero_gpu.astype(np.float64) - zero_ref
-    ztie = _half_dist(zpre.astype(np.float64)) < TIE_EPS
-    bad = ~((zdiff == 0) | ((np.abs(zdiff) == 1) & ztie))
-    assert not bad.any(), f"zero mismatch on tokens {np.flatnonzero(bad)[:8]}: {zero_gpu[bad][:4]} vs {zero_ref[bad][:4]}"
+    zpre64 = zpre.astype(np.float64)
+    zero_ok = (zdiff == 0) | (np.abs(zero_gpu - zpre64) <= 0.5 + w_zero)
+    bad = ~zero_ok
+    assert not bad.any(), (f"zero mismatch on tokens {np.flatnonzero(bad)[:8]}: "
+                           f"{zero_gpu[bad][:4]} vs {zero_ref[bad][:4]}")
     shifted = np.flatnonzero(zdiff != 0)
-    if shifted.size:  # the other side of a zero-point tie: redo the codes with the GPU's zero
-        y32 = y_ref.astype(np.float32)
-        for t in shifted:
-            v = np.rint(y32[t] / scale_ref[t]) + zero_gpu[t]
-            codes_ref[t] = np.clip(v, 0, 15).astype(np.uint8)
-            vpre[t] = y32[t] / scale_ref[t] + zero_gpu[t]
+    for t in shifted:  # the other side of a zero-point tie: redo the codes with the GPU's zero
+        v = np.rint(y32[t] / scale_ref[t]) + zero_gpu[t]
+        codes_ref[t] = np.clip(v, 0, 15).astype(np.uint8)
+        vpre[t] = y32[t] / scale_ref[t] + zero_gpu[t]
 
     diff = codes_gpu.astype(np.int32) - codes_ref.astype(np.int32)
     mism = diff != 0
-    tie = _half_dist(vpre.astype(np.float64)) < TIE_EPS
-    hard = mism & ~((np.abs(diff) == 1) & tie)
+    window = w_code[:, None]
+    tie = _half_dist(vpre.astype(np.float64)) < window
+    allowed_step = 1 + np.floor(window)
+    hard = mism & ~((np.abs(diff) <= allowed_step) & tie)
+    wide = window > 0.5  # rounding noise spans whole codes: judge by the dequantized value
+    if wide.any():
+        hard = hard & ~wide
     assert not hard.any(), (f"{int(hard.sum())} code mismatches away from ties, first at "
                             f"{np.argwhere(hard)[:4].tolist()}")
-    allowed = math.ceil(TIE_FRAC * T * n)
-    assert int(mism.sum()) <= allowed, f"{int(mism.sum())} tie mismatches > {allowed}"
-    return {"code_mismatches": int(mism.sum()), "zero_ties": int(shifted.size),
-            "scale_rel_max": float(srel.max()) if srel.size else 0.0}
+    well = w_code <= TIE_EPS
+    n_well = int(mism[well].sum())
+    allowed = math.ceil(TIE_FRAC * max(int(well.sum()), 1) * n)
+    assert n_well <= allowed, f"{n_well} tie mismatches on well-conditioned tokens > {allowed}"
+    if not strict:
+        deq = (codes_gpu.astype(np.float64) - zero_gpu[:, None]) * scale_gpu[:, None].astype(np.float64)
+        lo_g = (0 - zero_gpu.astype(np.float64)) * scale_gpu
+        hi_g = (15 - zero_gpu.astype(np.float64)) * scale_gpu
+        yc = np.clip(y_ref, lo_g[:, None], hi_g[:, None])
+        err = np.abs(deq - yc)
+        lim = scale_gpu[:, None] * 0.5 * (1 + 1e-5) + delta[:, None] + 1e-30
+        assert (err <= lim).all(), f"dequantized error {float((err - lim).max()):.3e} above half a step"
+    return {"code_mismatches": int(mism.sum()), "mismatch_frac": float(mism.mean()) if mism.size else 0.0,
+            "zero_ties": int(shifted.size), "scale_rel_max": float(srel.max()) if srel.size else 0.0,
+            "ill_conditioned_tokens": int((~well).sum())}
+
+
+def record(name: str, stats: dict) -> None:
+    """Append a test's parity statistics to $SIGNROT_PARITY_STATS (JSON lines), if set."""
+    path = os.environ.get("SIGNROT_PARITY_STATS")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": name, **stats}) + "\n")
