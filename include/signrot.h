@@ -77,6 +77,30 @@ signrot_status signrot_calibrate(const void* x, int32_t dtype, int64_t T, int32_
                                  int32_t* k_out, float* xk_out, void* stream);
 
 /*
+ * signrot_calibrate_static -- signrot_calibrate without a caller workspace. (Not from the SignRot
+ * pages, which have no counterpart: it exists for callers that cannot allocate device memory.)
+ *
+ * Some callers cannot hand the library an 8 * n byte device workspace: runtimes that reserve all
+ * device memory in one pool at start-up and forbid later cudaMalloc calls, plugins whose host
+ * framework owns the allocator and passes them only inputs and outputs, and latency-bound code
+ * that must not risk the device-wide synchronisation a cudaMalloc or cudaFree can cause. This call
+ * takes the same arguments as signrot_calibrate minus ws, and keeps the per-channel keys in a
+ * fixed array inside the library's device image (SIGNROT_STATIC_SCRATCH_MAX_N channels, 256 KB,
+ * held on every GPU that loads the library until the process exits). It allocates nothing.
+ *   - n > SIGNROT_STATIC_SCRATCH_MAX_N returns SIGNROT_ERR_UNSUPPORTED with a message.
+ *   - The first call on a device looks the array's device address up (cudaGetSymbolAddress with
+ *     that device current) and caches it; make that first call before any stream capture.
+ *   - All calls on a device share the one array, and it keeps the last call's contents:
+ *     accumulate == 0 clears it first; accumulate != 0 folds into whatever the previous call on
+ *     that device left there. Calls that overlap on the GPU (other streams, other host threads)
+ *     race on the array; serialise them.
+ */
+#define SIGNROT_STATIC_SCRATCH_MAX_N 32768
+signrot_status signrot_calibrate_static(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                        int64_t t_offset, int32_t accumulate, int32_t* k_out,
+                                        float* xk_out, void* stream);
+
+/*
  * signrot_build_sign -- the sign adjustment vector s.
  *
  * Follows the explainer's "SignRot asks one crowd to walk across the hall": every output j is

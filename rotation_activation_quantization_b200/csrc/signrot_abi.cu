@@ -393,3 +393,11 @@ const char* signrot_last_error(void) { return g_last_error; }
 uint64_t signrot_kernel_launches(void) { return signrot::g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"
+
+void signrot::set_last_error(const char* msg) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
+}
+
+extern "C" {
+
+}  // extern "C"

@@ -10,6 +10,9 @@ namespace signrot {
 // Counts every kernel launch the library issues (read by signrot_kernel_launches).
 void count_launch(int n = 1);
 
+// Sets the message signrot_last_error returns on this host thread.
+void set_last_error(const char* msg);
+
 // Library-owned Paley H_28 (paley_gf27.cpp), row-major, entries +/-1.
 void paley_h28(int8_t h[28][28]);
 

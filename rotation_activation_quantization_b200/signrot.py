@@ -23,6 +23,7 @@ _c_i32, _c_i64, _c_p, _c_f = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ct
 
 _SIGNATURES = {
     "signrot_calibrate": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_i64, _c_p, _c_i32, _c_p, _c_p, _c_p],
+    "signrot_calibrate_static": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_i64, _c_i32, _c_p, _c_p, _c_p],
     "signrot_build_sign": [_c_i32, _c_p, _c_p, _c_p, _c_p, _c_p],
     "signrot_rotate": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_i64, _c_p],
     "signrot_rotate_quant": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_i32, _c_f,
@@ -142,6 +143,21 @@ def calibrate(x: torch.Tensor, ws: torch.Tensor | None = None, accumulate: bool 
                                      int(bool(accumulate)), _ptr(k_out), _ptr(xk_out), _stream(dev, stream))
     _check("signrot_calibrate", st)
     return k_out, xk_out, ws
+
+
+def calibrate_static(x: torch.Tensor, accumulate: bool = False, t_offset: int = 0,
+                     k_out: torch.Tensor | None = None, xk_out: torch.Tensor | None = None, stream=None):
+    """calibrate() with the workspace kept in the library's fixed device array (no allocation by
+    the library; outputs are allocated here only when not passed). Returns (k, x_k)."""
+    T, n, ld = _rows(x)
+    dev = x.device
+    k_out = torch.empty(1, dtype=torch.int32, device=dev) if k_out is None else k_out
+    xk_out = torch.empty(1, dtype=torch.float32, device=dev) if xk_out is None else xk_out
+    with torch.cuda.device(dev):
+        st = lib().signrot_calibrate_static(_ptr(x), _dtype_code(x), T, n, ld, int(t_offset),
+                                            int(bool(accumulate)), _ptr(k_out), _ptr(xk_out), _stream(dev, stream))
+    _check("signrot_calibrate_static", st)
+    return k_out, xk_out
 
 
 def build_sign(n: int, k: torch.Tensor, xk: torch.Tensor, d: torch.Tensor,
