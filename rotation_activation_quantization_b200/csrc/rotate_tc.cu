@@ -53,13 +53,13 @@ namespace {
 
 using namespace ptx;
 
-// Eight warps, two per SM sub-partition, so each thread may hold up to 255 registers (each
-// sub-partition has a 16K-register file; a third warp on one would cap every thread at 168).
-constexpr int kThreads = 256;
-constexpr int kEpiWarps = 4;   // warps 0-3
-constexpr int kDWarps = 2;     // warps 4-5
-constexpr int kTmaWarp = 6;
-constexpr int kMmaWarp = 7;
+// Warp roles. Up to 128 columns per token the epilogue runs as two groups of four warps that
+// take alternate tokens (12 warps, 168 registers each: three warps share each SM sub-partition's
+// 16K-register file); at 256 columns a lane holds more values, so one group (8 warps, up to 255
+// registers). Each group's warp w reads TMEM lane quadrant w % 4.
+constexpr int kDWarps = 2;
+__host__ __device__ constexpr int epi_groups(int ncol) { return ncol <= 128 ? 2 : 1; }
+__host__ __device__ constexpr int threads_for(int ncol) { return 32 * (4 * epi_groups(ncol) + kDWarps + 2); }
 constexpr uint32_t kABytes = 128 * 128 * 2;  // A: 128 x 128 bf16
 constexpr uint32_t kBoxBytes = 16 * 128;     // one TMA box: 16 rows x 64 bf16 (128 B) = 2 KB
 constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23: fp32 whose ulp is 1
@@ -93,7 +93,7 @@ struct SignPlan {
   float sigma;
   int32_t c_k;       // F = 28: H_28 column of the outlier (g(a) = H_28[a][c_k])
   uint32_t e_hi;     // bits of the outlier index that index A's rows (h2 or r)
-  uint32_t e_lo;     // bits that index the TMEM columns: butterfly flips
+  uint32_t e_lo;     // bits that index the TMEM columns: applied as the column permutation b ^ e_lo
   bool active;
 };
 
@@ -156,14 +156,14 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 // ---------------------------------------------------------------------------- FWHT in registers
 
 // Butterfly on bit kBit of the column index over pairs p[i] = (w[2i], w[2i+1]).
-template <int kPairs, int kBit, bool kFlip>
+template <int kPairs, int kBit>
 __device__ __forceinline__ void fwht_stage(float2 (&p)[kPairs]) {
   if constexpr (kBit == 0) {
 #pragma unroll
     for (int i = 0; i < kPairs; ++i) {
       const float u = p[i].x, v = p[i].y;
       p[i].x = u + v;
-      p[i].y = kFlip ? v - u : u - v;
+      p[i].y = u - v;
     }
   } else {
     constexpr int hs = 1 << (kBit - 1);
@@ -172,42 +172,85 @@ __device__ __forceinline__ void fwht_stage(float2 (&p)[kPairs]) {
       if ((i & hs) == 0) {
         const float2 u = p[i], v = p[i + hs];
         p[i] = __fadd2_rn(u, v);
-        p[i + hs] = kFlip ? fsub2(v, u) : fsub2(u, v);
+        p[i + hs] = fsub2(u, v);
       }
     }
   }
 }
 
-template <int kPairs, int kBit>
-__device__ __forceinline__ void fwht_stage_rt(float2 (&p)[kPairs], uint32_t flips) {
-  if ((flips >> kBit) & 1u)
-    fwht_stage<kPairs, kBit, true>(p);
-  else
-    fwht_stage<kPairs, kBit, false>(p);
-}
-
 // All stages over kBits bits of the in-thread column index.
 template <int kPairs, int kBits>
-__device__ __forceinline__ void fwht_local(float2 (&p)[kPairs], uint32_t flips) {
-  fwht_stage_rt<kPairs, 0>(p, flips);
-  if (kBits > 1) fwht_stage_rt<kPairs, (kBits > 1 ? 1 : 0)>(p, flips);
-  if (kBits > 2) fwht_stage_rt<kPairs, (kBits > 2 ? 2 : 0)>(p, flips);
-  if (kBits > 3) fwht_stage_rt<kPairs, (kBits > 3 ? 3 : 0)>(p, flips);
-  if (kBits > 4) fwht_stage_rt<kPairs, (kBits > 4 ? 4 : 0)>(p, flips);
-  if (kBits > 5) fwht_stage_rt<kPairs, (kBits > 5 ? 5 : 0)>(p, flips);
-  if (kBits > 6) fwht_stage_rt<kPairs, (kBits > 6 ? 6 : 0)>(p, flips);
+__device__ __forceinline__ void fwht_local(float2 (&p)[kPairs]) {
+  fwht_stage<kPairs, 0>(p);
+  if constexpr (kBits > 1) fwht_stage<kPairs, 1>(p);
+  if constexpr (kBits > 2) fwht_stage<kPairs, 2>(p);
+  if constexpr (kBits > 3) fwht_stage<kPairs, 3>(p);
+  if constexpr (kBits > 4) fwht_stage<kPairs, 4>(p);
+  if constexpr (kBits > 5) fwht_stage<kPairs, 5>(p);
+  if constexpr (kBits > 6) fwht_stage<kPairs, 6>(p);
+}
+
+// The D pass's column permutation within one 16-byte segment: element m moves to m ^ kF
+// (words by kF >> 1, the two bf16 halves of each word by kF & 1).
+template <int kF>
+__device__ __forceinline__ uint4 permute_segment(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t t = w[i ^ (kF >> 1)];
+    o[i] = (kF & 1) ? __byte_perm(t, 0, 0x1032) : t;
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// One stage of the D pass: apply D's sign masks to every 16-byte chunk and move it to the slot
+// (chunk ^ seg_xor) of the same 128-byte row, permuting its 8 columns by kF.
+template <int kF, int kStageChunks, int kDThreads>
+__device__ __forceinline__ void d_pass_stage(uint4* base, const uint4* masks, int td, uint32_t seg_xor) {
+#pragma unroll 2
+  for (int c0 = 0; c0 < kStageChunks; c0 += 4 * kDThreads) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int ch = c0 + u * kDThreads + td;
+      if (ch < kStageChunks) {
+        v[u] = base[ch];
+        const uint4 m = masks[ch];
+        v[u].x ^= m.x;
+        v[u].y ^= m.y;
+        v[u].z ^= m.z;
+        v[u].w ^= m.w;
+      }
+    }
+    __syncwarp();  // a row's 8 chunks are read by 8 lanes of this warp before any is rewritten
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int ch = c0 + u * kDThreads + td;
+      if (ch < kStageChunks) base[ch ^ static_cast<int>(seg_xor)] = permute_segment<kF>(v[u]);
+    }
+    __syncwarp();
+  }
 }
 
 // TMEM -> registers: kN pairs (2 * kN consecutive columns from taddr) into p[kOff .. kOff + kN).
 template <int kOff, int kN, int kPairs>
 __device__ __forceinline__ void tmem_load_pairs(uint32_t taddr, float2 (&p)[kPairs]) {
   static_assert(kN % 16 == 0 && kOff + kN <= kPairs, "whole 32-column loads only");
+  if constexpr (kN == 64) {
+    uint32_t r[128];
+    tmem_ld128(taddr, r);
 #pragma unroll
-  for (int c = 0; c < kN; c += 16) {
-    uint32_t r[32];
-    tmem_ld32(taddr + 2 * c, r);
+    for (int i = 0; i < 64; ++i) p[kOff + i] = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+  } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) p[kOff + c + i] = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+    for (int c = 0; c < kN; c += 16) {
+      uint32_t r[32];
+      tmem_ld32(taddr + 2 * c, r);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        p[kOff + c + i] = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+    }
   }
 }
 
@@ -228,7 +271,15 @@ __device__ __forceinline__ void tmem_store_pairs(uint32_t taddr, const float2 (&
 
 // Elementwise general sign vector: bit r of sbits flips the sign of column r.
 template <int kPairs>
-__device__ __forceinline__ void apply_sign_bits(float2 (&p)[kPairs], const uint32_t* sbits) {
+__device__ __forceinline__ void apply_sign_bits(float2 (&p)[kPairs], const uint32_t* sbits_in) {
+  // The words are the same for every token; hiding that from the compiler keeps it from hoisting
+  // all 2*kPairs masks out of the token loop into registers.
+  uint32_t sbits[(2 * kPairs + 31) / 32];
+#pragma unroll
+  for (int w = 0; w < (2 * kPairs + 31) / 32; ++w) {
+    sbits[w] = sbits_in[w];
+    asm volatile("" : "+r"(sbits[w]));
+  }
 #pragma unroll
   for (int i = 0; i < kPairs; ++i) {
     const int r0 = 2 * i, r1 = 2 * i + 1;
@@ -266,13 +317,14 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&u)[8]) {
   return __byte_perm(w0, w1, 0x5410);
 }
 
-// Quantize kPairs pairs (consecutive columns) into packed words (kPairs / 4 of them).
-template <int kPairs, bool kClamp>
-__device__ __forceinline__ void quant_pack(const float2 (&p)[kPairs], float c, float zm, uint32_t* words) {
+// Quantize 16 pairs (32 consecutive columns) into one 16-byte store of packed nibbles.
+template <bool kClamp>
+__device__ __forceinline__ uint4 quant16(const float2* p, float c, float zm) {
   const float2 c2 = make_float2(c, c), z2 = make_float2(zm, zm);
   const float lo_m = kMagic, hi_m = kMagic + 15.f;
+  uint32_t words[4];
 #pragma unroll
-  for (int g = 0; g < kPairs / 4; ++g) {
+  for (int g = 0; g < 4; ++g) {
     uint32_t u[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -286,20 +338,21 @@ __device__ __forceinline__ void quant_pack(const float2 (&p)[kPairs], float c, f
     }
     words[g] = pack8(u);
   }
+  return make_uint4(words[0], words[1], words[2], words[3]);
 }
 
 // Quantize + store one run of 2*kPairs consecutive channels at q_out (16 B aligned).
 template <int kPairs>
 __device__ __forceinline__ void quant_store(const float2 (&p)[kPairs], float c, float zm, bool clamp,
                                             uint8_t* q_out) {
-  uint32_t words[kPairs / 4];
-  if (clamp)
-    quant_pack<kPairs, true>(p, c, zm, words);
-  else
-    quant_pack<kPairs, false>(p, c, zm, words);
   uint4* dst = reinterpret_cast<uint4*>(q_out);
+  if (clamp) {
 #pragma unroll
-  for (int i = 0; i < kPairs / 16; ++i) dst[i] = make_uint4(words[4 * i], words[4 * i + 1], words[4 * i + 2], words[4 * i + 3]);
+    for (int i = 0; i < kPairs / 16; ++i) dst[i] = quant16<true>(p + 16 * i, c, zm);
+  } else {
+#pragma unroll
+    for (int i = 0; i < kPairs / 16; ++i) dst[i] = quant16<false>(p + 16 * i, c, zm);
+  }
 }
 
 template <int kPairs>
@@ -337,7 +390,7 @@ __device__ __forceinline__ TokenGrid token_grid(float lo_w, float hi_w, float rs
 // ------------------------------------------------------------------------------------- kernel
 
 template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
-__global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcParams p) {
+__global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcParams p) {
   constexpr int kKRows = kF28 ? 112 : 128;     // K of the MMA chain
   constexpr int kKSteps = kKRows / 16;
   constexpr int kChunksN = kNcol / 64;          // 64-column TMA / swizzle atoms per token
@@ -349,6 +402,13 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
   constexpr int kStageChunks = kChunksN * kKRows * 8;  // 16-B chunks per stage
   constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                               (static_cast<uint32_t>(kNcol >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+  constexpr int kGroups = epi_groups(kNcol);
+  constexpr int kEpiWarps = 4 * kGroups;  // warps [0, kEpiWarps): epilogue
+  constexpr int kTmaWarp = kEpiWarps + kDWarps;  // then the D-pass warps, TMA, MMA
+  constexpr int kMmaWarp = kTmaWarp + 1;
+  constexpr int kThreads = threads_for(kNcol);
+  constexpr int kTBufs = 2 * kGroups;  // TMEM accumulators in flight
+  static_assert(kTBufs * kNcol <= 512, "TMEM holds 512 columns");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -361,13 +421,20 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
   uint64_t* dready = bars + S;
   uint64_t* empty = bars + 2 * S;
   uint64_t* tfull = bars + 3 * S;
-  uint64_t* tempty = bars + 3 * S + 2;
-  uint64_t* redbar = bars + 3 * S + 4;  // the 4 epilogue warps' min/max exchange, per TMEM buffer
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 6);
-  float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [2 buffers][4 warps][lo, hi]
+  uint64_t* tempty = bars + 3 * S + kTBufs;
+  uint64_t* redbar = bars + 3 * S + 2 * kTBufs;  // a group's min/max exchange, per TMEM buffer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 3 * kTBufs);
+  float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [buffer][4 quadrants][lo, hi]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SignPlan sp = make_plan<kF28, kNcol>(p);
+  // The outlier-channel sign's column factor (-1)^popcount(b & e_lo) is applied as a column
+  // permutation of the MMA's input (diag(h_e) H = H P_e, P_e: b -> b ^ e): TMEM column b then
+  // holds input column b ^ e_lo. Bits >= 6 pick the 64-column TMA box, bits 3-5 the 16-byte
+  // slot the D pass writes, bits 0-2 the D pass's in-segment register permutation.
+  const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
+  const uint32_t seg_xor = (col_xor >> 3) & 7u;
+  const int box_xor = static_cast<int>(col_xor >> 6);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -375,10 +442,10 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
       mbar_init(smem_u32(&dready[i]), kDWarps);
       mbar_init(smem_u32(&empty[i]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kTBufs; ++i) {
       mbar_init(smem_u32(&tfull[i]), 1);
-      mbar_init(smem_u32(&tempty[i]), kEpiWarps);
-      mbar_init(smem_u32(&redbar[i]), kEpiWarps);
+      mbar_init(smem_u32(&tempty[i]), 4);  // the 4 warps of the group that owns buffer i
+      mbar_init(smem_u32(&redbar[i]), 4);
     }
     fence_mbar_init();
   }
@@ -393,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
   for (int ch = threadIdx.x; ch < kStageChunks; ch += kThreads) {
     const int nb = ch / (kKRows * 8), rem = ch % (kKRows * 8);
     const int row = rem >> 3, slot = rem & 7;
-    const int b0 = nb * 64 + ((slot ^ (row & 7)) << 3);
+    const int b0 = (nb ^ box_xor) * 64 + ((slot ^ (row & 7)) << 3);
     const int j0 = kF28 ? (row >> 2) * M + (row & 3) * kNcol + b0 : row * kNcol + b0;
 #pragma unroll
     for (int w = 0; w < 4; ++w)
@@ -426,9 +493,9 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
           for (int bx = 0; bx < kBoxesPerChunk; ++bx) {
             const uint32_t dst = dst0 + nb * kChunkBytes + bx * kBoxBytes;
             if (kF28)
-              tma_load_4d(dst, &tmap, nb * 64, 0, bx * 4, t, fb);
+              tma_load_4d(dst, &tmap, (nb ^ box_xor) * 64, 0, bx * 4, t, fb);
             else
-              tma_load_3d(dst, &tmap, nb * 64, bx * 16, t, fb);
+              tma_load_3d(dst, &tmap, (nb ^ box_xor) * 64, bx * 16, t, fb);
           }
         }
       }
@@ -443,9 +510,9 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
       const uint32_t a_base = smem_u32(a_smem);
       int i = 0;
       for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
-        const int st = i % S, tb = i & 1;
+        const int st = i % S, tb = i % kTBufs;
         if (!mbar_wait(smem_u32(&dready[st]), (i / S) & 1)) { flag_error(); break; }
-        if (!mbar_wait(smem_u32(&tempty[tb]), ((i >> 1) & 1) ^ 1)) { flag_error(); break; }
+        if (!mbar_wait(smem_u32(&tempty[tb]), ((i / kTBufs) & 1) ^ 1)) { flag_error(); break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + tb * kNcol;
         const uint32_t b_base = smem_u32(ring + st * kStageBytes);
@@ -459,10 +526,10 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
         mma_commit(smem_u32(&tfull[tb]));
       }
       // leave no MMA in flight behind: the last commit must have landed before TMEM is freed
-      if (i > 0 && !mbar_wait(smem_u32(&tfull[(i - 1) & 1]), ((i - 1) >> 1) & 1)) flag_error();
+      if (i > 0 && !mbar_wait(smem_u32(&tfull[(i - 1) % kTBufs]), ((i - 1) / kTBufs) & 1)) flag_error();
     }
   } else if (warp >= kEpiWarps) {
-    // ------------------------------------------------------------------ D pass (warps 4-5)
+    // ------------------------------------------------------------------ D pass (2 warps)
     const int td = threadIdx.x - kEpiWarps * 32;
     const uint4* masks = reinterpret_cast<const uint4*>(dmask);
     int i = 0;
@@ -470,23 +537,24 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
       const int st = i % S;
       if (!mbar_wait(smem_u32(&full[st]), (i / S) & 1)) { flag_error(); break; }
       uint4* base = reinterpret_cast<uint4*>(ring + st * kStageBytes);
-#pragma unroll 4
-      for (int ch = td; ch < kStageChunks; ch += kDWarps * 32) {
-        uint4 v = base[ch];
-        const uint4 m = masks[ch];
-        v.x ^= m.x;
-        v.y ^= m.y;
-        v.z ^= m.z;
-        v.w ^= m.w;
-        base[ch] = v;
+      constexpr int kDT = kDWarps * 32;
+      switch (col_xor & 7u) {  // low three bits of the column permutation, fixed per launch
+        case 0: d_pass_stage<0, kStageChunks, kDT>(base, masks, td, seg_xor); break;
+        case 1: d_pass_stage<1, kStageChunks, kDT>(base, masks, td, seg_xor); break;
+        case 2: d_pass_stage<2, kStageChunks, kDT>(base, masks, td, seg_xor); break;
+        case 3: d_pass_stage<3, kStageChunks, kDT>(base, masks, td, seg_xor); break;
+        case 4: d_pass_stage<4, kStageChunks, kDT>(base, masks, td, seg_xor); break;
+        case 5: d_pass_stage<5, kStageChunks, kDT>(base, masks, td, seg_xor); break;
+        case 6: d_pass_stage<6, kStageChunks, kDT>(base, masks, td, seg_xor); break;
+        default: d_pass_stage<7, kStageChunks, kDT>(base, masks, td, seg_xor); break;
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&dready[st]));
     }
   } else {
-    // ------------------------------------------------------------------ epilogue (warps 0-3)
-    const int quad = warp;
+    // ------------------------------------------------------------------ epilogue
+    const int quad = warp & 3, group = warp >> 2;
     const bool active = !kF28 || lane < 28;
     // this lane's output run: row (h2' = quad, a = lane) or r = quad * 32 + lane
     const int64_t j0 = kF28 ? static_cast<int64_t>(lane) * M + quad * kNcol : static_cast<int64_t>(quad * 32 + lane) * kNcol;
@@ -500,12 +568,12 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
         sbits[w] = b;
       }
     }
-    const uint32_t flips = sp.active ? sp.e_lo : 0u;
     const float rs = p.inv_sqrt_n;
-    int i = 0;
-    for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
-      const int tb = i & 1;
-      if (!mbar_wait(smem_u32(&tfull[tb]), (i >> 1) & 1)) { flag_error(); break; }
+    // this group takes every kGroups-th of the CTA's tokens, starting at its index
+    int i = group;
+    for (int t = blockIdx.x + group * gridDim.x; t < p.T; t += kGroups * gridDim.x, i += kGroups) {
+      const int tb = i % kTBufs;
+      if (!mbar_wait(smem_u32(&tfull[tb]), (i / kTBufs) & 1)) { flag_error(); break; }
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tb * kNcol;
       float2 v[kPairs];
@@ -515,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&tempty[tb]));
-        fwht_local<kPairs, (kNcol == 64 ? 6 : 7)>(v, flips);
+        fwht_local<kPairs, (kNcol == 64 ? 6 : 7)>(v);
         if (kVecSign) apply_sign_bits<kPairs>(v, sbits);
         if (active) local_minmax<kPairs>(v, lo, hi);
       } else {
@@ -523,10 +591,9 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
           tmem_load_pairs<0, kPairs>(taddr + hh * 128, v);
-          fwht_local<kPairs, 7>(v, flips);
+          fwht_local<kPairs, 7>(v);
           tmem_store_pairs<kPairs>(taddr + hh * 128, v);
         }
-        const bool f7 = (flips >> 7) & 1u;
 #pragma unroll 1
         for (int g = 0; g < 2; ++g) {
           float2 u[32];
@@ -536,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
           for (int k = 0; k < 32; ++k) {
             const float2 a = v[k], b = u[k];
             v[k] = __fadd2_rn(a, b);
-            v[32 + k] = f7 ? fsub2(b, a) : fsub2(a, b);
+            v[32 + k] = fsub2(a, b);
           }
           if (kVecSign) {
             const uint32_t sb[2] = {sbits[2 * g], sbits[2 * g + 1]};
@@ -564,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&redbar[tb]));
-      if (!mbar_wait(smem_u32(&redbar[tb]), (i >> 1) & 1)) { flag_error(); break; }
+      if (!mbar_wait(smem_u32(&redbar[tb]), (i / kTBufs) & 1)) { flag_error(); break; }
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         lo = fminf(lo, red[(tb * 4 + w) * 2]);
@@ -572,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
       }
       if (kQuant) {
         const TokenGrid g = token_grid(lo, hi, rs, p.clip);
-        if (threadIdx.x == 0) {
+        if (quad == 0 && lane == 0) {
           p.scale[t] = g.scale;
           p.zero[t] = g.zero;
         }
@@ -580,7 +647,6 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
         if constexpr (kNcol <= 128) {
           if (active) quant_store<kPairs>(v, g.c, g.zm, g.clamp, qrow + (j0 >> 1));
         } else {
-          const bool f7 = (flips >> 7) & 1u;
 #pragma unroll 1
           for (int gg = 0; gg < 2; ++gg) {
             float2 u[32], lo_half[32], hi_half[32];
@@ -590,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
             for (int k = 0; k < 32; ++k) {
               const float2 a = lo_half[k], b = u[k];
               lo_half[k] = __fadd2_rn(a, b);
-              hi_half[k] = f7 ? fsub2(b, a) : fsub2(a, b);
+              hi_half[k] = fsub2(a, b);
             }
             if (kVecSign) {
               const uint32_t sb[2] = {sbits[2 * gg], sbits[2 * gg + 1]};
@@ -609,7 +675,6 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
         if constexpr (kNcol <= 128) {
           if (active) store_y<kPairs>(v, rs, yrow + j0);
         } else {
-          const bool f7 = (flips >> 7) & 1u;
 #pragma unroll 1
           for (int gg = 0; gg < 2; ++gg) {
             float2 u[32], lo_half[32], hi_half[32];
@@ -619,7 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1) rotq_tc_kernel(const __grid_const
             for (int k = 0; k < 32; ++k) {
               const float2 a = lo_half[k], b = u[k];
               lo_half[k] = __fadd2_rn(a, b);
-              hi_half[k] = f7 ? fsub2(b, a) : fsub2(a, b);
+              hi_half[k] = fsub2(a, b);
             }
             if (kVecSign) {
               const uint32_t sb[2] = {sbits[2 * gg], sbits[2 * gg + 1]};
@@ -682,7 +747,7 @@ cudaError_t launch_tc(const CUtensorMap& tmap, const TcParams& p0, cudaStream_t 
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int grid = p.T < sms ? p.T : sms;
-  kern<<<grid, kThreads, smem, st>>>(tmap, p);
+  kern<<<grid, threads_for(kNcol), smem, st>>>(tmap, p);
   count_launch();
   return cudaGetLastError();
 }
