@@ -68,6 +68,8 @@ constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23: fp32 whose ulp is 1
 __device__ __forceinline__ void flag_error(unsigned int bit = 1u) { atomicOr(&g_device_error, bit); }
 
 struct TcParams {
+  const void* xraw;  // rows, for the streamed variant's bulk copies
+  int64_t ldx;
   int32_t T;
   int32_t n;
   int32_t logM;  // F = 28: M = 2^logM; F = 1: unused
@@ -230,6 +232,53 @@ __device__ __forceinline__ void d_pass_stage(uint4* base, const uint4* masks, in
       if (ch < kStageChunks) base[ch ^ static_cast<int>(seg_xor)] = permute_segment<kF>(v[u]);
     }
     __syncwarp();
+  }
+}
+
+// D's 8 signs of one 16-byte chunk, packed so that (bits << w) & 0x80008000 is the XOR mask of
+// word w: the sign of element 2w sits at bit 15 - w, that of element 2w + 1 at bit 31 - w.
+__device__ __forceinline__ uint32_t chunk_sign_bits(uint2 d8) {
+  uint32_t b = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const uint32_t byte = ((e < 4 ? d8.x : d8.y) >> (8 * (e & 3))) & 0xffu;
+    b |= ((byte >> 7) & 1u) << (15 + 16 * (e & 1) - (e >> 1));
+  }
+  return b;
+}
+
+__device__ __forceinline__ uint4 apply_chunk_signs(uint4 v, uint32_t bits) {
+  v.x ^= bits & 0x80008000u;
+  v.y ^= (bits << 1) & 0x80008000u;
+  v.z ^= (bits << 2) & 0x80008000u;
+  v.w ^= (bits << 3) & 0x80008000u;
+  return v;
+}
+
+// Streamed D pass for one token: each thread takes its kPerD fixed 16-byte chunks of the linear
+// row, flips D's sign bits, permutes the 8 columns by kF and stores the chunk at its place in the
+// swizzled MMA tile. Chunks go in batches of kBatch loads, then kBatch stores: the two buffers
+// are different, but the compiler cannot know it and would otherwise wait out every load.
+template <int kF, int kPerD, int kDT, int kBatch>
+__device__ __forceinline__ void stream_d_pass(const uint4* src, uint8_t* tile, const uint32_t (&bits_in)[kPerD],
+                                              const uint32_t (&dst)[kPerD], int td) {
+  static_assert(kPerD % kBatch == 0, "whole batches");
+  // The sign words are the same for every token; hiding that from the compiler keeps it from
+  // hoisting the four expanded masks per chunk out of the token loop into registers.
+  uint32_t bits[kPerD];
+#pragma unroll
+  for (int u = 0; u < kPerD; ++u) {
+    bits[u] = bits_in[u];
+    asm volatile("" : "+r"(bits[u]));
+  }
+#pragma unroll
+  for (int u0 = 0; u0 < kPerD; u0 += kBatch) {
+    uint4 v[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) v[b] = src[td + kDT * (u0 + b)];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b)
+      *reinterpret_cast<uint4*>(tile + dst[u0 + b]) = permute_segment<kF>(apply_chunk_signs(v[b], bits[u0 + b]));
   }
 }
 
@@ -411,7 +460,9 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_tc_kernel(const __
   static_assert(kTBufs * kNcol <= 512, "TMEM holds 512 columns");
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base for the 128-byte swizzle atoms; offsetting the pointer (not casting
+  // through an integer) keeps the compiler's knowledge that every access below is to shared memory
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int S = p.stages;
   uint8_t* a_smem = smem;
   uint32_t* dmask = reinterpret_cast<uint32_t*>(smem + kABytes);  // D sign masks, stage layout
@@ -715,6 +766,249 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_tc_kernel(const __
   }
 }
 
+// ------------------------------------------------------------- streamed variant (<= 128 columns)
+//
+// The same pipeline with the token row fetched as ONE contiguous bulk copy into a linear shared-
+// memory ring (the tensor-map boxes above gather 16 separate 128-byte pieces each, which streams
+// ~14% slower from HBM). The D-pass warps then do the whole layout change in one read and one
+// write per 16-byte chunk: linear row -> XOR D -> column permutation -> the MMA's swizzled tile,
+// with each thread's D masks and destinations held in registers. Tiles are double-buffered, and
+// the producer starts streaming before the A matrix and the masks are built.
+
+template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
+__global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_stream_kernel(TcParams p) {
+  static_assert(kNcol <= 128, "the streamed variant keeps a token's lane line in registers");
+  constexpr int kKRows = kF28 ? 112 : 128;
+  constexpr int kKSteps = kKRows / 16;
+  constexpr int kChunksN = kNcol / 64;
+  constexpr uint32_t kChunkBytes = kKRows * 128;
+  constexpr uint32_t kRowBytes = kChunksN * kChunkBytes;  // = 2n: one bf16 token row
+  constexpr int kRowChunks = static_cast<int>(kRowBytes / 16);
+  constexpr int kDT = kDWarps * 32;
+  constexpr int kPerD = kRowChunks / kDT;
+  static_assert(kRowChunks % kDT == 0, "D-pass threads own whole chunks");
+  constexpr int kDBatch = kPerD % 7 == 0 ? 7 : (kPerD % 8 == 0 ? 8 : kPerD);
+  constexpr int kPairs = kNcol / 2;
+  constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                              (static_cast<uint32_t>(kNcol >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+  constexpr int kGroups = epi_groups(kNcol);
+  constexpr int kEpiWarps = 4 * kGroups;
+  constexpr int kTmaWarp = kEpiWarps + kDWarps;
+  constexpr int kMmaWarp = kTmaWarp + 1;
+  constexpr int kThreads = threads_for(kNcol);
+  constexpr int kTBufs = 2 * kGroups;
+  constexpr uint32_t kTmemCols = kTBufs * kNcol < 32 ? 32 : kTBufs * kNcol;
+  static_assert(kTBufs * kNcol <= 512, "TMEM holds 512 columns");
+
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned base for the 128-byte swizzle atoms; offsetting the pointer (not casting
+  // through an integer) keeps the compiler's knowledge that every access below is to shared memory
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int S = p.stages;
+  uint8_t* a_smem = smem;
+  uint8_t* btile = smem + kABytes;             // 2 swizzled MMA tiles
+  uint8_t* lin = btile + 2 * kRowBytes;        // S linear rows
+  uint64_t* bars = reinterpret_cast<uint64_t*>(lin + S * kRowBytes);
+  uint64_t* lfull = bars;
+  uint64_t* lempty = bars + S;
+  uint64_t* bfull = bars + 2 * S;
+  uint64_t* bempty = bars + 2 * S + 2;
+  uint64_t* tfull = bars + 2 * S + 4;
+  uint64_t* tempty = tfull + kTBufs;
+  uint64_t* redbar = tempty + kTBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redbar + kTBufs);
+  float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [buffer][4 quadrants][lo, hi]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(&lfull[i]), 1);
+      mbar_init(smem_u32(&lempty[i]), kDWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bfull[i]), kDWarps);
+      mbar_init(smem_u32(&bempty[i]), 1);
+    }
+    for (int i = 0; i < kTBufs; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), 4);
+      mbar_init(smem_u32(&redbar[i]), 4);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------------ producer: one row per copy
+    if (lane == 0) {
+      const char* x = static_cast<const char*>(p.xraw);
+      int i = 0;
+      for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+        const int st = i % S;
+        if (!mbar_wait(smem_u32(&lempty[st]), ((i / S) & 1) ^ 1)) { flag_error(); break; }
+        const uint32_t fb = smem_u32(&lfull[st]);
+        mbar_arrive_expect_tx(fb, kRowBytes);
+        bulk_load(smem_u32(lin + st * kRowBytes), x + static_cast<int64_t>(t) * p.ldx * 2, kRowBytes, fb);
+      }
+      const int issued = i;
+      for (int j = issued - S > 0 ? issued - S : 0; j < issued; ++j)
+        if (!mbar_wait(smem_u32(&lfull[j % S]), (j / S) & 1)) { flag_error(); break; }
+    }
+    tc_fence_before();
+    __syncthreads();
+    return;
+  }
+
+  // everyone else: A, the sign plan, TMEM, then the roles
+  const SignPlan sp = make_plan<kF28, kNcol>(p);
+  const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
+  const int ntid = threadIdx.x < kTmaWarp * 32 ? threadIdx.x : threadIdx.x - 32;
+  for (int idx = ntid; idx < 128 * 128; idx += kThreads - 32) {
+    const int m = idx >> 7, k = idx & 127;
+    *reinterpret_cast<uint16_t*>(a_smem + a_offset(m, k)) = a_entry<kF28>(m, k, sp, p.h);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  asm volatile("bar.sync 1, %0;" ::"r"(kThreads - 32) : "memory");
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int M = kF28 ? (1 << p.logM) : 0;
+
+  if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t a_base = smem_u32(a_smem);
+      int i = 0;
+      for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+        const int bb = i & 1, tb = i % kTBufs;
+        if (!mbar_wait(smem_u32(&bfull[bb]), (i >> 1) & 1)) { flag_error(); break; }
+        if (!mbar_wait(smem_u32(&tempty[tb]), ((i / kTBufs) & 1) ^ 1)) { flag_error(); break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + tb * kNcol;
+        const uint32_t b_base = smem_u32(btile + bb * kRowBytes);
+#pragma unroll
+        for (int ks = 0; ks < kKSteps; ++ks) {
+          const uint64_t ad = smem_desc(a_base + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc(b_base + ks * 2048, kChunkBytes, 1024);
+          mma_bf16(d_tmem, ad, bd, kIdesc, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&bempty[bb]));
+        mma_commit(smem_u32(&tfull[tb]));
+      }
+      if (i > 0 && !mbar_wait(smem_u32(&tfull[(i - 1) % kTBufs]), ((i - 1) / kTBufs) & 1)) flag_error();
+    }
+  } else if (warp >= kEpiWarps) {
+    // ------------------------------------------------------------------ D pass: linear -> tile
+    const int td = threadIdx.x - kEpiWarps * 32;
+    uint32_t bits[kPerD];
+    uint32_t dst[kPerD];
+#pragma unroll
+    for (int u = 0; u < kPerD; ++u) {
+      const int L = td + kDT * u;
+      const int k = L / (kNcol / 8), b0 = (L % (kNcol / 8)) * 8;
+      const int j0 = kF28 ? (k >> 2) * M + (k & 3) * kNcol + b0 : k * kNcol + b0;
+      bits[u] = chunk_sign_bits(*reinterpret_cast<const uint2*>(p.d + j0));  // 8 signs, 8-byte aligned
+      const int bp = b0 ^ static_cast<int>(col_xor & ~7u);  // where this chunk's columns go
+      const int nbp = bp >> 6, segp = (bp >> 3) & 7;
+      dst[u] = static_cast<uint32_t>(nbp) * kChunkBytes + k * 128 + ((segp ^ (k & 7)) << 4);
+    }
+    int i = 0;
+    for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+      const int st = i % S, bb = i & 1;
+      if (!mbar_wait(smem_u32(&lfull[st]), (i / S) & 1)) { flag_error(); break; }
+      if (!mbar_wait(smem_u32(&bempty[bb]), ((i >> 1) & 1) ^ 1)) { flag_error(); break; }
+      const uint4* src = reinterpret_cast<const uint4*>(lin + st * kRowBytes);
+      uint8_t* tile = btile + bb * kRowBytes;
+      switch (col_xor & 7u) {
+        case 0: stream_d_pass<0, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
+        case 1: stream_d_pass<1, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
+        case 2: stream_d_pass<2, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
+        case 3: stream_d_pass<3, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
+        case 4: stream_d_pass<4, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
+        case 5: stream_d_pass<5, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
+        case 6: stream_d_pass<6, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
+        default: stream_d_pass<7, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&lempty[st]));
+        mbar_arrive(smem_u32(&bfull[bb]));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int quad = warp & 3, group = warp >> 2;
+    const bool active = !kF28 || lane < 28;
+    const int64_t j0 = kF28 ? static_cast<int64_t>(lane) * M + quad * kNcol : static_cast<int64_t>(quad * 32 + lane) * kNcol;
+    uint32_t sbits[kVecSign ? kNcol / 32 : 1];
+    if (kVecSign) {
+#pragma unroll
+      for (int w = 0; w < kNcol / 32; ++w) {
+        uint32_t b = 0;
+        if (active)
+          for (int r = 0; r < 32; ++r) b |= (p.s[j0 + 32 * w + r] < 0 ? 1u : 0u) << r;
+        sbits[w] = b;
+      }
+    }
+    const float rs = p.inv_sqrt_n;
+    int i = group;
+    for (int t = blockIdx.x + group * gridDim.x; t < p.T; t += kGroups * gridDim.x, i += kGroups) {
+      const int tb = i % kTBufs;
+      if (!mbar_wait(smem_u32(&tfull[tb]), (i / kTBufs) & 1)) { flag_error(); break; }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tb * kNcol;
+      float2 v[kPairs];
+      tmem_load_pairs<0, kPairs>(taddr, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty[tb]));
+      fwht_local<kPairs, (kNcol == 64 ? 6 : 7)>(v);
+      if (kVecSign) apply_sign_bits<kPairs>(v, sbits);
+      float lo = pos_inf(), hi = -pos_inf();
+      if (active) local_minmax<kPairs>(v, lo, hi);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      }
+      if (lane == 0) {
+        red[(tb * 4 + quad) * 2] = lo;
+        red[(tb * 4 + quad) * 2 + 1] = hi;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&redbar[tb]));
+      if (!mbar_wait(smem_u32(&redbar[tb]), (i / kTBufs) & 1)) { flag_error(); break; }
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        lo = fminf(lo, red[(tb * 4 + w) * 2]);
+        hi = fmaxf(hi, red[(tb * 4 + w) * 2 + 1]);
+      }
+      if (kQuant) {
+        const TokenGrid g = token_grid(lo, hi, rs, p.clip);
+        if (quad == 0 && lane == 0) {
+          p.scale[t] = g.scale;
+          p.zero[t] = g.zero;
+        }
+        if (active) quant_store<kPairs>(v, g.c, g.zm, g.clamp, p.q + static_cast<int64_t>(t) * (p.n >> 1) + (j0 >> 1));
+      } else if (active) {
+        store_y<kPairs>(v, rs, p.y + static_cast<int64_t>(t) * p.ldy + j0);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------------------------- host
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -752,6 +1046,34 @@ cudaError_t launch_tc(const CUtensorMap& tmap, const TcParams& p0, cudaStream_t 
   return cudaGetLastError();
 }
 
+template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
+cudaError_t launch_stream(const TcParams& p0, cudaStream_t st) {
+  constexpr int kKRows = kF28 ? 112 : 128;
+  constexpr uint32_t kRowBytes = (kNcol / 64) * kKRows * 128;
+  constexpr uint32_t kSmemBudget = 227 * 1024 - 1024 - kABytes - 2 * kRowBytes - 512;
+  TcParams p = p0;
+  p.stages = static_cast<int>(kSmemBudget / kRowBytes);
+  if (p.stages > 8) p.stages = 8;
+  const size_t smem = 1024 + kABytes + 2 * kRowBytes + static_cast<size_t>(p.stages) * kRowBytes + 512;
+  auto kern = rotq_stream_kernel<kNcol, kF28, kVecSign, kQuant>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = p.T < sms ? p.T : sms;
+  kern<<<grid, threads_for(kNcol), smem, st>>>(p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <int kNcol, bool kF28>
+cudaError_t dispatch_stream(const TcParams& p, bool vec_sign, bool quant, cudaStream_t st) {
+  if (vec_sign)
+    return quant ? launch_stream<kNcol, kF28, true, true>(p, st) : launch_stream<kNcol, kF28, true, false>(p, st);
+  return quant ? launch_stream<kNcol, kF28, false, true>(p, st) : launch_stream<kNcol, kF28, false, false>(p, st);
+}
+
 template <int kNcol, bool kF28>
 cudaError_t dispatch_mode(const CUtensorMap& tmap, const TcParams& p, bool vec_sign, bool quant, cudaStream_t st) {
   if (vec_sign)
@@ -770,9 +1092,35 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
   const bool quant = a.q != nullptr;
   if (quant && reinterpret_cast<uintptr_t>(a.q) % 16 != 0) return cudaErrorNotSupported;
   if (!quant && (reinterpret_cast<uintptr_t>(a.y) % 16 != 0 || a.ldy % 4 != 0)) return cudaErrorNotSupported;
+  TcParams p{};
+  p.xraw = a.x;
+  p.ldx = a.ld;
+  p.T = static_cast<int32_t>(a.T);
+  p.n = a.shape.n;
+  p.logM = a.shape.logM;
+  p.d = a.d;
+  p.s = a.s;
+  p.kp = a.kp;
+  p.xkp = a.xkp;
+  p.q = a.q;
+  p.scale = a.scale;
+  p.zero = a.zero;
+  p.y = a.y;
+  p.ldy = a.ldy;
+  p.clip = a.clip;
+  p.inv_sqrt_n = a.inv_sqrt_n;
+  p.h = h;
+  const bool vec = a.s != nullptr && a.kp == nullptr;
+  // Streamed variant where a D-pass thread's masks fit in registers: 28 chunks per thread at
+  // M = 512 with the 28-block factor, 16 or 14 at 64 columns. A 128-column power-of-two row
+  // (32 chunks per thread) and 256-column rows take the tensor-map kernel.
+  if (reinterpret_cast<uintptr_t>(a.d) % 8 == 0) {
+    if (ncol == 64) return f28 ? dispatch_stream<64, true>(p, vec, quant, st) : dispatch_stream<64, false>(p, vec, quant, st);
+    if (ncol == 128 && f28) return dispatch_stream<128, true>(p, vec, quant, st);
+  }
+
   auto encode = encode_fn();
   if (encode == nullptr) return cudaErrorNotSupported;
-
   CUtensorMap tmap;
   CUresult r;
   const cuuint32_t elem_strides[4] = {1, 1, 1, 1};
@@ -794,24 +1142,6 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   }
   if (r != CUDA_SUCCESS) return cudaErrorNotSupported;
-
-  TcParams p{};
-  p.T = static_cast<int32_t>(a.T);
-  p.n = a.shape.n;
-  p.logM = a.shape.logM;
-  p.d = a.d;
-  p.s = a.s;
-  p.kp = a.kp;
-  p.xkp = a.xkp;
-  p.q = a.q;
-  p.scale = a.scale;
-  p.zero = a.zero;
-  p.y = a.y;
-  p.ldy = a.ldy;
-  p.clip = a.clip;
-  p.inv_sqrt_n = a.inv_sqrt_n;
-  p.h = h;
-  const bool vec = a.s != nullptr && a.kp == nullptr;
   if (f28) {
     if (ncol == 64) return dispatch_mode<64, true>(tmap, p, vec, quant, st);
     if (ncol == 128) return dispatch_mode<128, true>(tmap, p, vec, quant, st);
