@@ -235,50 +235,41 @@ __device__ __forceinline__ void d_pass_stage(uint4* base, const uint4* masks, in
   }
 }
 
-// D's 8 signs of one 16-byte chunk, packed so that (bits << w) & 0x80008000 is the XOR mask of
-// word w: the sign of element 2w sits at bit 15 - w, that of element 2w + 1 at bit 31 - w.
-__device__ __forceinline__ uint32_t chunk_sign_bits(uint2 d8) {
-  uint32_t b = 0;
+// D's signs of one 16-byte chunk (8 bf16 columns) as XOR masks on its four 32-bit words.
+__device__ __forceinline__ uint4 chunk_sign_masks(uint2 d8) {
+  uint32_t w[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const uint32_t byte = ((e < 4 ? d8.x : d8.y) >> (8 * (e & 3))) & 0xffu;
-    b |= ((byte >> 7) & 1u) << (15 + 16 * (e & 1) - (e >> 1));
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t pair = ((i < 2 ? d8.x : d8.y) >> (16 * (i & 1))) & 0xffffu;  // d[2i], d[2i+1]
+    w[i] = ((pair & 0x80u) << 8) | ((pair & 0x8000u) << 16);
   }
-  return b;
+  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__device__ __forceinline__ uint4 apply_chunk_signs(uint4 v, uint32_t bits) {
-  v.x ^= bits & 0x80008000u;
-  v.y ^= (bits << 1) & 0x80008000u;
-  v.z ^= (bits << 2) & 0x80008000u;
-  v.w ^= (bits << 3) & 0x80008000u;
-  return v;
-}
-
-// Streamed D pass for one token: each thread takes its kPerD fixed 16-byte chunks of the linear
-// row, flips D's sign bits, permutes the 8 columns by kF and stores the chunk at its place in the
-// swizzled MMA tile. Chunks go in batches of kBatch loads, then kBatch stores: the two buffers
-// are different, but the compiler cannot know it and would otherwise wait out every load.
-template <int kF, int kPerD, int kDT, int kBatch>
-__device__ __forceinline__ void stream_d_pass(const uint4* src, uint8_t* tile, const uint32_t (&bits_in)[kPerD],
-                                              const uint32_t (&dst)[kPerD], int td) {
-  static_assert(kPerD % kBatch == 0, "whole batches");
-  // The sign words are the same for every token; hiding that from the compiler keeps it from
-  // hoisting the four expanded masks per chunk out of the token loop into registers.
-  uint32_t bits[kPerD];
-#pragma unroll
-  for (int u = 0; u < kPerD; ++u) {
-    bits[u] = bits_in[u];
-    asm volatile("" : "+r"(bits[u]));
-  }
+// Streamed D pass for one token: each lane takes its kPerD fixed 16-byte chunks of the linear row
+// (32 chunks apart; the last one only when `last` is set), flips D's signs, moves the chunk's words
+// by kW (the permutation's bits 1 and 2; bit 0 is left to the epilogue) and stores the chunk at its
+// place in the swizzled MMA tile. Chunks go in batches of kBatch loads, then kBatch stores: the
+// two buffers are different, but the compiler cannot know it and would otherwise wait out every
+// load.
+template <int kW, int kPerD, int kBatch>
+__device__ __forceinline__ void stream_d_pass(const uint4* src, uint8_t* tile, const uint4 (&mask)[kPerD],
+                                              const uint32_t (&dst)[kPerD], bool last) {
 #pragma unroll
   for (int u0 = 0; u0 < kPerD; u0 += kBatch) {
-    uint4 v[kBatch];
+    constexpr int kB = kBatch;
+    uint4 v[kB];
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) v[b] = src[td + kDT * (u0 + b)];
+    for (int b = 0; b < kB; ++b)
+      if (u0 + b < kPerD && (u0 + b < kPerD - 1 || last)) v[b] = src[32 * (u0 + b)];
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b)
-      *reinterpret_cast<uint4*>(tile + dst[u0 + b]) = permute_segment<kF>(apply_chunk_signs(v[b], bits[u0 + b]));
+    for (int b = 0; b < kB; ++b) {
+      if (u0 + b < kPerD && (u0 + b < kPerD - 1 || last)) {
+        const uint4 m = mask[u0 + b];
+        const uint32_t w[4] = {v[b].x ^ m.x, v[b].y ^ m.y, v[b].z ^ m.z, v[b].w ^ m.w};
+        *reinterpret_cast<uint4*>(tile + dst[u0 + b]) = make_uint4(w[kW], w[1 ^ kW], w[2 ^ kW], w[3 ^ kW]);
+      }
+    }
   }
 }
 
@@ -339,6 +330,27 @@ __device__ __forceinline__ void apply_sign_bits(float2 (&p)[kPairs], const uint3
   }
 }
 
+// Extremes of the even (.x) and odd (.y) columns kept apart, so that a sign flip of every odd
+// column can be applied to the result instead of the values.
+template <int kPairs>
+__device__ __forceinline__ void local_minmax_xy(const float2 (&p)[kPairs], float& lx, float& hx, float& ly, float& hy) {
+  float l0 = p[0].x, h0 = p[0].x, l1 = p[0].y, h1 = p[0].y;
+#pragma unroll
+  for (int i = 1; i + 1 < kPairs; i += 2) {
+    l0 = fmin3(l0, p[i].x, p[i + 1].x);
+    h0 = fmax3(h0, p[i].x, p[i + 1].x);
+    l1 = fmin3(l1, p[i].y, p[i + 1].y);
+    h1 = fmax3(h1, p[i].y, p[i + 1].y);
+  }
+  if ((kPairs & 1) == 0) {
+    l0 = fminf(l0, p[kPairs - 1].x);
+    h0 = fmaxf(h0, p[kPairs - 1].x);
+    l1 = fminf(l1, p[kPairs - 1].y);
+    h1 = fmaxf(h1, p[kPairs - 1].y);
+  }
+  lx = l0; hx = h0; ly = l1; hy = h1;
+}
+
 template <int kPairs>
 __device__ __forceinline__ void local_minmax(const float2 (&p)[kPairs], float& lo, float& hi) {
   float l0 = p[0].x, l1 = p[0].y, h0 = p[0].x, h1 = p[0].y;
@@ -368,8 +380,8 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&u)[8]) {
 
 // Quantize 16 pairs (32 consecutive columns) into one 16-byte store of packed nibbles.
 template <bool kClamp>
-__device__ __forceinline__ uint4 quant16(const float2* p, float c, float zm) {
-  const float2 c2 = make_float2(c, c), z2 = make_float2(zm, zm);
+__device__ __forceinline__ uint4 quant16(const float2* p, float2 c2, float zm) {
+  const float2 z2 = make_float2(zm, zm);
   const float lo_m = kMagic, hi_m = kMagic + 15.f;
   uint32_t words[4];
 #pragma unroll
@@ -390,26 +402,31 @@ __device__ __forceinline__ uint4 quant16(const float2* p, float c, float zm) {
   return make_uint4(words[0], words[1], words[2], words[3]);
 }
 
-// Quantize + store one run of 2*kPairs consecutive channels at q_out (16 B aligned).
+// Quantize + store one run of 2*kPairs consecutive channels at q_out (16 B aligned); c2 holds the
+// multipliers of the even and the odd channels.
 template <int kPairs>
-__device__ __forceinline__ void quant_store(const float2 (&p)[kPairs], float c, float zm, bool clamp,
+__device__ __forceinline__ void quant_store(const float2 (&p)[kPairs], float2 c2, float zm, bool clamp,
                                             uint8_t* q_out) {
   uint4* dst = reinterpret_cast<uint4*>(q_out);
   if (clamp) {
 #pragma unroll
-    for (int i = 0; i < kPairs / 16; ++i) dst[i] = quant16<true>(p + 16 * i, c, zm);
+    for (int i = 0; i < kPairs / 16; ++i) dst[i] = quant16<true>(p + 16 * i, c2, zm);
   } else {
 #pragma unroll
-    for (int i = 0; i < kPairs / 16; ++i) dst[i] = quant16<false>(p + 16 * i, c, zm);
+    for (int i = 0; i < kPairs / 16; ++i) dst[i] = quant16<false>(p + 16 * i, c2, zm);
   }
 }
 
 template <int kPairs>
-__device__ __forceinline__ void store_y(const float2 (&p)[kPairs], float rs, float* y_out) {
+__device__ __forceinline__ void store_y(const float2 (&p)[kPairs], float rs, float* y_out, float rs_odd) {
   float4* dst = reinterpret_cast<float4*>(y_out);
 #pragma unroll
   for (int i = 0; i < kPairs / 2; ++i)
-    dst[i] = make_float4(p[2 * i].x * rs, p[2 * i].y * rs, p[2 * i + 1].x * rs, p[2 * i + 1].y * rs);
+    dst[i] = make_float4(p[2 * i].x * rs, p[2 * i].y * rs_odd, p[2 * i + 1].x * rs, p[2 * i + 1].y * rs_odd);
+}
+template <int kPairs>
+__device__ __forceinline__ void store_y(const float2 (&p)[kPairs], float rs, float* y_out) {
+  store_y<kPairs>(p, rs, y_out, rs);
 }
 
 struct TokenGrid {
@@ -696,7 +713,7 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_tc_kernel(const __
         }
         uint8_t* qrow = p.q + static_cast<int64_t>(t) * (p.n >> 1);
         if constexpr (kNcol <= 128) {
-          if (active) quant_store<kPairs>(v, g.c, g.zm, g.clamp, qrow + (j0 >> 1));
+          if (active) quant_store<kPairs>(v, make_float2(g.c, g.c), g.zm, g.clamp, qrow + (j0 >> 1));
         } else {
 #pragma unroll 1
           for (int gg = 0; gg < 2; ++gg) {
@@ -716,8 +733,8 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_tc_kernel(const __
               apply_sign_bits<32>(hi_half, sb2);
             }
             if (active) {
-              quant_store<32>(lo_half, g.c, g.zm, g.clamp, qrow + ((j0 + gg * 64) >> 1));
-              quant_store<32>(hi_half, g.c, g.zm, g.clamp, qrow + ((j0 + 128 + gg * 64) >> 1));
+              quant_store<32>(lo_half, make_float2(g.c, g.c), g.zm, g.clamp, qrow + ((j0 + gg * 64) >> 1));
+              quant_store<32>(hi_half, make_float2(g.c, g.c), g.zm, g.clamp, qrow + ((j0 + 128 + gg * 64) >> 1));
             }
           }
         }
@@ -768,15 +785,27 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_tc_kernel(const __
 
 // ------------------------------------------------------------- streamed variant (<= 128 columns)
 //
-// The same pipeline with the token row fetched as ONE contiguous bulk copy into a linear shared-
+// mbar_wait by every lane of the warp, with one verdict for all of them (a lane whose wait ran out
+// makes the whole warp leave its loop together).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+
+// The same pipeline with the token row fetched by plain 1-D bulk copies into a linear shared-
 // memory ring (the tensor-map boxes above gather 16 separate 128-byte pieces each, which streams
-// ~14% slower from HBM). The D-pass warps then do the whole layout change in one read and one
-// write per 16-byte chunk: linear row -> XOR D -> column permutation -> the MMA's swizzled tile,
-// with each thread's D masks and destinations held in registers. Tiles are double-buffered, and
-// the producer starts streaming before the A matrix and the masks are built.
+// ~14% slower from HBM). Three D-pass warps each own a third of the row: they stream it in with
+// their own bulk copies and do the whole layout change in one read and one write per 16-byte chunk
+// (linear row -> XOR D -> column permutation -> the MMA's swizzled tile), with their D sign masks
+// and destinations held in registers, refilling their part of a ring slot as soon as they have
+// converted it. A fourth warp issues the MMAs; three tiles let the D warps run two tokens ahead of
+// it. Twelve warps in all: a thirteenth would cap every thread at 128 registers.
+
+constexpr int kStreamDWarps = 3;
+constexpr int kStreamTiles = 3;
+__host__ __device__ constexpr int stream_threads(int ncol) { return 32 * (4 * epi_groups(ncol) + kStreamDWarps + 1); }
 
 template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
-__global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_stream_kernel(TcParams p) {
+__global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(TcParams p) {
   static_assert(kNcol <= 128, "the streamed variant keeps a token's lane line in registers");
   constexpr int kKRows = kF28 ? 112 : 128;
   constexpr int kKSteps = kKRows / 16;
@@ -784,19 +813,21 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_stream_kernel(TcPa
   constexpr uint32_t kChunkBytes = kKRows * 128;
   constexpr uint32_t kRowBytes = kChunksN * kChunkBytes;  // = 2n: one bf16 token row
   constexpr int kRowChunks = static_cast<int>(kRowBytes / 16);
-  constexpr int kDT = kDWarps * 32;
-  constexpr int kPerD = kRowChunks / kDT;
-  static_assert(kRowChunks % kDT == 0, "D-pass threads own whole chunks");
-  constexpr int kDBatch = kPerD % 7 == 0 ? 7 : (kPerD % 8 == 0 ? 8 : kPerD);
+  constexpr int kDW = kStreamDWarps;
+  constexpr int kLaneChunks = kRowChunks / 32;             // chunks per lane position, over all D warps
+  static_assert(kRowChunks % 32 == 0, "D-pass lanes own whole chunks");
+  constexpr int kPerD = (kLaneChunks + kDW - 1) / kDW;     // D warp w: kPerD or kPerD - 1 per lane
+  constexpr int kDBatch = 7;
   constexpr int kPairs = kNcol / 2;
   constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                               (static_cast<uint32_t>(kNcol >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
   constexpr int kGroups = epi_groups(kNcol);
-  constexpr int kEpiWarps = 4 * kGroups;
-  constexpr int kTmaWarp = kEpiWarps + kDWarps;
-  constexpr int kMmaWarp = kTmaWarp + 1;
-  constexpr int kThreads = threads_for(kNcol);
+  constexpr int kEpiWarps = 4 * kGroups;  // warps [0, kEpiWarps): epilogue
+  constexpr int kDWarp0 = kEpiWarps;      // then the D warps and the MMA warp
+  constexpr int kMmaWarp = kDWarp0 + kDW;
+  constexpr int kThreads = stream_threads(kNcol);
   constexpr int kTBufs = 2 * kGroups;
+  constexpr int kTiles = kStreamTiles;
   constexpr uint32_t kTmemCols = kTBufs * kNcol < 32 ? 32 : kTBufs * kNcol;
   static_assert(kTBufs * kNcol <= 512, "TMEM holds 512 columns");
 
@@ -806,64 +837,59 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_stream_kernel(TcPa
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int S = p.stages;
   uint8_t* a_smem = smem;
-  uint8_t* btile = smem + kABytes;             // 2 swizzled MMA tiles
-  uint8_t* lin = btile + 2 * kRowBytes;        // S linear rows
+  uint8_t* btile = smem + kABytes;             // kTiles swizzled MMA tiles
+  uint8_t* lin = btile + kTiles * kRowBytes;   // S linear rows
   uint64_t* bars = reinterpret_cast<uint64_t*>(lin + S * kRowBytes);
-  uint64_t* lfull = bars;
-  uint64_t* lempty = bars + S;
-  uint64_t* bfull = bars + 2 * S;
-  uint64_t* bempty = bars + 2 * S + 2;
-  uint64_t* tfull = bars + 2 * S + 4;
+  uint64_t* lfull = bars;                      // [slot][D warp]
+  uint64_t* bfull = bars + S * kDW;            // [tile]
+  uint64_t* bempty = bfull + kTiles;
+  uint64_t* tfull = bempty + kTiles;           // [TMEM buffer]
   uint64_t* tempty = tfull + kTBufs;
-  uint64_t* redbar = tempty + kTBufs;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redbar + kTBufs);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + kTBufs);
   float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [buffer][4 quadrants][lo, hi]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) {
-      mbar_init(smem_u32(&lfull[i]), 1);
-      mbar_init(smem_u32(&lempty[i]), kDWarps);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bfull[i]), kDWarps);
+    for (int i = 0; i < S * kDW; ++i) mbar_init(smem_u32(&lfull[i]), 1);
+    for (int i = 0; i < kTiles; ++i) {
+      mbar_init(smem_u32(&bfull[i]), kDW);
       mbar_init(smem_u32(&bempty[i]), 1);
     }
     for (int i = 0; i < kTBufs; ++i) {
       mbar_init(smem_u32(&tfull[i]), 1);
       mbar_init(smem_u32(&tempty[i]), 4);
-      mbar_init(smem_u32(&redbar[i]), 4);
     }
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == kTmaWarp) {
-    // ------------------------------------------------------------------ producer: one row per copy
-    if (lane == 0) {
-      const char* x = static_cast<const char*>(p.xraw);
-      int i = 0;
-      for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
-        const int st = i % S;
-        if (!mbar_wait(smem_u32(&lempty[st]), ((i / S) & 1) ^ 1)) { flag_error(); break; }
-        const uint32_t fb = smem_u32(&lfull[st]);
-        mbar_arrive_expect_tx(fb, kRowBytes);
-        bulk_load(smem_u32(lin + st * kRowBytes), x + static_cast<int64_t>(t) * p.ldx * 2, kRowBytes, fb);
-      }
-      const int issued = i;
-      for (int j = issued - S > 0 ? issued - S : 0; j < issued; ++j)
-        if (!mbar_wait(smem_u32(&lfull[j % S]), (j / S) & 1)) { flag_error(); break; }
+  // D warp w's share of the row: lane chunks [c0, c0 + 32 * per) of the kRowChunks
+  const bool dwarp = warp >= kDWarp0 && warp < kMmaWarp;
+  const int dw = dwarp ? warp - kDWarp0 : 0;
+  const int per = kLaneChunks / kDW + (dw < kLaneChunks % kDW ? 1 : 0);
+  const int c0 = 32 * (dw * (kLaneChunks / kDW) + (dw < kLaneChunks % kDW ? dw : kLaneChunks % kDW));
+  const uint32_t part_bytes = static_cast<uint32_t>(per) * 32u * 16u;
+  const char* xpart = static_cast<const char*>(p.xraw) + c0 * 16;
+  // one D warp's copy of its share of token t into ring slot st
+  auto stream_in = [&](int st, int t) {
+    const uint32_t fb = smem_u32(&lfull[st * kDW + dw]);
+    mbar_arrive_expect_tx(fb, part_bytes);
+    bulk_load(smem_u32(lin + st * kRowBytes + c0 * 16), xpart + static_cast<int64_t>(t) * p.ldx * 2, part_bytes, fb);
+  };
+  int issued = 0;  // bulk copies this D warp has started (lane 0)
+  if (dwarp && lane == 0) {
+    // start streaming before the A matrix and the masks are built
+    for (int st = 0; st < S; ++st) {
+      const int t = blockIdx.x + st * gridDim.x;
+      if (t >= p.T) break;
+      stream_in(st, t);
+      ++issued;
     }
-    tc_fence_before();
-    __syncthreads();
-    return;
   }
 
-  // everyone else: A, the sign plan, TMEM, then the roles
   const SignPlan sp = make_plan<kF28, kNcol>(p);
   const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
-  const int ntid = threadIdx.x < kTmaWarp * 32 ? threadIdx.x : threadIdx.x - 32;
-  for (int idx = ntid; idx < 128 * 128; idx += kThreads - 32) {
+  for (int idx = threadIdx.x; idx < 128 * 128; idx += kThreads) {
     const int m = idx >> 7, k = idx & 127;
     *reinterpret_cast<uint16_t*>(a_smem + a_offset(m, k)) = a_entry<kF28>(m, k, sp, p.h);
   }
@@ -873,7 +899,7 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_stream_kernel(TcPa
   }
   fence_proxy_async_smem();
   tc_fence_before();
-  asm volatile("bar.sync 1, %0;" ::"r"(kThreads - 32) : "memory");
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int M = kF28 ? (1 << p.logM) : 0;
@@ -884,9 +910,12 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_stream_kernel(TcPa
       const uint32_t a_base = smem_u32(a_smem);
       int i = 0;
       for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
-        const int bb = i & 1, tb = i % kTBufs;
-        if (!mbar_wait(smem_u32(&bfull[bb]), (i >> 1) & 1)) { flag_error(); break; }
-        if (!mbar_wait(smem_u32(&tempty[tb]), ((i / kTBufs) & 1) ^ 1)) { flag_error(); break; }
+        const int bb = i % kTiles, tb = i % kTBufs;
+        if (!mbar_wait(smem_u32(&bfull[bb]), (i / kTiles) & 1) ||
+            !mbar_wait(smem_u32(&tempty[tb]), ((i / kTBufs) & 1) ^ 1)) {
+          flag_error();
+          break;
+        }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + tb * kNcol;
         const uint32_t b_base = smem_u32(btile + bb * kRowBytes);
@@ -899,46 +928,57 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_stream_kernel(TcPa
         mma_commit(smem_u32(&bempty[bb]));
         mma_commit(smem_u32(&tfull[tb]));
       }
+      // the last MMAs finish before the TMEM is freed
       if (i > 0 && !mbar_wait(smem_u32(&tfull[(i - 1) % kTBufs]), ((i - 1) / kTBufs) & 1)) flag_error();
     }
-  } else if (warp >= kEpiWarps) {
+  } else if (dwarp) {
     // ------------------------------------------------------------------ D pass: linear -> tile
-    const int td = threadIdx.x - kEpiWarps * 32;
-    uint32_t bits[kPerD];
+    const bool last = per == kPerD;  // this warp also takes its lanes' kPerD-th chunk
+    uint4 mask[kPerD];
     uint32_t dst[kPerD];
 #pragma unroll
     for (int u = 0; u < kPerD; ++u) {
-      const int L = td + kDT * u;
+      const int L = (u < per ? c0 + 32 * u : c0) + lane;
       const int k = L / (kNcol / 8), b0 = (L % (kNcol / 8)) * 8;
       const int j0 = kF28 ? (k >> 2) * M + (k & 3) * kNcol + b0 : k * kNcol + b0;
-      bits[u] = chunk_sign_bits(*reinterpret_cast<const uint2*>(p.d + j0));  // 8 signs, 8-byte aligned
+      mask[u] = chunk_sign_masks(*reinterpret_cast<const uint2*>(p.d + j0));  // 8 signs, 8-byte aligned
       const int bp = b0 ^ static_cast<int>(col_xor & ~7u);  // where this chunk's columns go
       const int nbp = bp >> 6, segp = (bp >> 3) & 7;
       dst[u] = static_cast<uint32_t>(nbp) * kChunkBytes + k * 128 + ((segp ^ (k & 7)) << 4);
     }
     int i = 0;
     for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
-      const int st = i % S, bb = i & 1;
-      if (!mbar_wait(smem_u32(&lfull[st]), (i / S) & 1)) { flag_error(); break; }
-      if (!mbar_wait(smem_u32(&bempty[bb]), ((i >> 1) & 1) ^ 1)) { flag_error(); break; }
-      const uint4* src = reinterpret_cast<const uint4*>(lin + st * kRowBytes);
-      uint8_t* tile = btile + bb * kRowBytes;
-      switch (col_xor & 7u) {
-        case 0: stream_d_pass<0, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
-        case 1: stream_d_pass<1, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
-        case 2: stream_d_pass<2, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
-        case 3: stream_d_pass<3, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
-        case 4: stream_d_pass<4, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
-        case 5: stream_d_pass<5, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
-        case 6: stream_d_pass<6, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
-        default: stream_d_pass<7, kPerD, kDT, kDBatch>(src, tile, bits, dst, td); break;
+      const int st = i % S, bb = i % kTiles;
+      if (!warp_wait(smem_u32(&lfull[st * kDW + dw]), (i / S) & 1) ||
+          !warp_wait(smem_u32(&bempty[bb]), ((i / kTiles) & 1) ^ 1)) {
+        flag_error();
+        break;
       }
+      const uint4* src = reinterpret_cast<const uint4*>(lin + st * kRowBytes) + c0 + lane;
+      uint8_t* tile = btile + bb * kRowBytes;
+      switch ((col_xor >> 1) & 3u) {
+        case 0: stream_d_pass<0, kPerD, kDBatch>(src, tile, mask, dst, last); break;
+        case 1: stream_d_pass<1, kPerD, kDBatch>(src, tile, mask, dst, last); break;
+        case 2: stream_d_pass<2, kPerD, kDBatch>(src, tile, mask, dst, last); break;
+        default: stream_d_pass<3, kPerD, kDBatch>(src, tile, mask, dst, last); break;
+      }
+      // the tile writes must reach the MMA (async proxy), and this slot's reads must be done
+      // before the next bulk copy overwrites it
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(smem_u32(&lempty[st]));
         mbar_arrive(smem_u32(&bfull[bb]));
+        const int tn = t + S * gridDim.x;
+        if (tn < p.T) {
+          stream_in(st, tn);
+          ++issued;
+        }
       }
+    }
+    if (lane == 0) {
+      // on an early exit, let this warp's copies still in flight land before the CTA ends
+      for (int j = i; j < issued; ++j)
+        if (!mbar_wait(smem_u32(&lfull[(j % S) * kDW + dw]), (j / S) & 1)) { flag_error(); break; }
     }
   } else {
     // ------------------------------------------------------------------ epilogue
@@ -956,10 +996,23 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_stream_kernel(TcPa
       }
     }
     const float rs = p.inv_sqrt_n;
+    // the outlier permutation's bit 0 is not applied to the input: every odd column of the
+    // transform comes out negated (H P_1 = diag((-1)^j) H), which min/max and quantization undo
+    const bool odd_neg = (col_xor & 1u) != 0;
+    // A warp whose wait runs out stops working but keeps taking its group's barrier, once per token
+    // like the others, so that no warp of the group is left waiting there.
+    bool live = true;
     int i = group;
     for (int t = blockIdx.x + group * gridDim.x; t < p.T; t += kGroups * gridDim.x, i += kGroups) {
       const int tb = i % kTBufs;
-      if (!mbar_wait(smem_u32(&tfull[tb]), (i / kTBufs) & 1)) { flag_error(); break; }
+      if (live && !warp_wait(smem_u32(&tfull[tb]), (i / kTBufs) & 1)) {
+        flag_error();
+        live = false;
+      }
+      if (!live) {
+        named_barrier_sync(1 + group, 128);
+        continue;
+      }
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tb * kNcol;
       float2 v[kPairs];
@@ -970,19 +1023,19 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_stream_kernel(TcPa
       fwht_local<kPairs, (kNcol == 64 ? 6 : 7)>(v);
       if (kVecSign) apply_sign_bits<kPairs>(v, sbits);
       float lo = pos_inf(), hi = -pos_inf();
-      if (active) local_minmax<kPairs>(v, lo, hi);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      if (active) {
+        float lx, hx, ly, hy;
+        local_minmax_xy<kPairs>(v, lx, hx, ly, hy);
+        lo = fminf(lx, odd_neg ? -hy : ly);
+        hi = fmaxf(hx, odd_neg ? -ly : hy);
       }
+      lo = warp_min(lo);
+      hi = warp_max(hi);
       if (lane == 0) {
         red[(tb * 4 + quad) * 2] = lo;
         red[(tb * 4 + quad) * 2 + 1] = hi;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&redbar[tb]));
-      if (!mbar_wait(smem_u32(&redbar[tb]), (i / kTBufs) & 1)) { flag_error(); break; }
+      named_barrier_sync(1 + group, 128);  // the group's four quadrant extremes are in
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         lo = fminf(lo, red[(tb * 4 + w) * 2]);
@@ -994,9 +1047,11 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_stream_kernel(TcPa
           p.scale[t] = g.scale;
           p.zero[t] = g.zero;
         }
-        if (active) quant_store<kPairs>(v, g.c, g.zm, g.clamp, p.q + static_cast<int64_t>(t) * (p.n >> 1) + (j0 >> 1));
+        if (active)
+          quant_store<kPairs>(v, make_float2(g.c, odd_neg ? -g.c : g.c), g.zm, g.clamp,
+                              p.q + static_cast<int64_t>(t) * (p.n >> 1) + (j0 >> 1));
       } else if (active) {
-        store_y<kPairs>(v, rs, p.y + static_cast<int64_t>(t) * p.ldy + j0);
+        store_y<kPairs>(v, rs, p.y + static_cast<int64_t>(t) * p.ldy + j0, odd_neg ? -rs : rs);
       }
     }
   }
@@ -1050,11 +1105,12 @@ template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
 cudaError_t launch_stream(const TcParams& p0, cudaStream_t st) {
   constexpr int kKRows = kF28 ? 112 : 128;
   constexpr uint32_t kRowBytes = (kNcol / 64) * kKRows * 128;
-  constexpr uint32_t kSmemBudget = 227 * 1024 - 1024 - kABytes - 2 * kRowBytes - 512;
+  constexpr uint32_t kSmemBudget = 227 * 1024 - 1024 - kABytes - kStreamTiles * kRowBytes - 1024;
   TcParams p = p0;
   p.stages = static_cast<int>(kSmemBudget / kRowBytes);
   if (p.stages > 8) p.stages = 8;
-  const size_t smem = 1024 + kABytes + 2 * kRowBytes + static_cast<size_t>(p.stages) * kRowBytes + 512;
+  if (p.stages < 2) return cudaErrorNotSupported;
+  const size_t smem = 1024 + kABytes + kStreamTiles * kRowBytes + static_cast<size_t>(p.stages) * kRowBytes + 1024;
   auto kern = rotq_stream_kernel<kNcol, kF28, kVecSign, kQuant>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -1062,7 +1118,7 @@ cudaError_t launch_stream(const TcParams& p0, cudaStream_t st) {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int grid = p.T < sms ? p.T : sms;
-  kern<<<grid, threads_for(kNcol), smem, st>>>(p);
+  kern<<<grid, stream_threads(kNcol), smem, st>>>(p);
   count_launch();
   return cudaGetLastError();
 }
@@ -1111,12 +1167,11 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
   p.inv_sqrt_n = a.inv_sqrt_n;
   p.h = h;
   const bool vec = a.s != nullptr && a.kp == nullptr;
-  // Streamed variant where a D-pass thread's masks fit in registers: 28 chunks per thread at
-  // M = 512 with the 28-block factor, 16 or 14 at 64 columns. A 128-column power-of-two row
-  // (32 chunks per thread) and 256-column rows take the tensor-map kernel.
+  // Streamed variant for rows of up to 128 columns per token (D read 8 bytes at a time); 256-column
+  // rows, whose lane lines do not fit in registers at once, take the tensor-map kernel.
   if (reinterpret_cast<uintptr_t>(a.d) % 8 == 0) {
     if (ncol == 64) return f28 ? dispatch_stream<64, true>(p, vec, quant, st) : dispatch_stream<64, false>(p, vec, quant, st);
-    if (ncol == 128 && f28) return dispatch_stream<128, true>(p, vec, quant, st);
+    if (ncol == 128) return f28 ? dispatch_stream<128, true>(p, vec, quant, st) : dispatch_stream<128, false>(p, vec, quant, st);
   }
 
   auto encode = encode_fn();
