@@ -86,7 +86,7 @@ def recorded_traffic(w: syn.Workload, digest: str):
         return None
     with open(p) as f:
         rec = json.load(f)
-    e = rec.get(f"config{w.index}")
+    e = rec.get(w.name)
     if not e or e.get("kernel_sources") != digest:
         return None
     return float(e["dram_bytes_per_token"]) * w.T
