@@ -438,18 +438,35 @@ struct TokenGrid {
 };
 
 __device__ __forceinline__ TokenGrid token_grid(float lo_w, float hi_w, float rs, float clip) {
+  // The grid sits on every token's critical path, so it avoids the second IEEE division: scale is
+  // the exact fp32 quotient (u - l) / 15; zero = rne(-l / scale) comes from -l * (1 / scale),
+  // which lies within a few ulps of the exact fp32 quotient -- only when that puts it within a
+  // guard band of a half-integer could the two round differently, and only then is the exact
+  // division taken. 1 / scale itself (for the codes) is the hardware approximation.
   const float lo_y = __fmul_rn(lo_w, rs), hi_y = __fmul_rn(hi_w, rs);
-  const QuantGrid g = make_grid(lo_y, hi_y, clip);
+  const float l = __fmul_rn(lo_y, clip), u = __fmul_rn(hi_y, clip);
   TokenGrid tg;
-  tg.scale = g.scale;
-  tg.zero = g.zero;
-  tg.c = __fmul_rn(rs, g.inv);
-  tg.zm = __fadd_rn(g.zero, kMagic);
+  float inv;
+  if (u == l) {
+    tg.scale = 1.f;
+    tg.zero = rintf(-l);
+    inv = 1.f;
+  } else {
+    tg.scale = __fdiv_rn(__fsub_rn(u, l), 15.f);
+    asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(tg.scale));
+    const float q0 = __fmul_rn(-l, inv);
+    tg.zero = rintf(q0);
+    const float off = fabsf(__fsub_rn(q0, tg.zero));      // distance to the nearest integer
+    const float guard = fmaf(fabsf(q0), 0x1p-19f, 0x1p-40f);  // ~16 ulps of q0
+    if (!(0.5f - off > guard)) tg.zero = rintf(__fdiv_rn(-l, tg.scale));
+  }
+  tg.c = __fmul_rn(rs, inv);
+  tg.zm = __fadd_rn(tg.zero, kMagic);
   // codes are monotone in w, so the row's extremes decide whether any code needs clamping;
   // a zero-point too large for the 1.5 * 2^23 trick also takes the clamped path
   const int c_lo = static_cast<int>(__float_as_uint(fmaf(lo_w, tg.c, tg.zm)) - __float_as_uint(kMagic));
   const int c_hi = static_cast<int>(__float_as_uint(fmaf(hi_w, tg.c, tg.zm)) - __float_as_uint(kMagic));
-  tg.clamp = !(c_lo >= 0 && c_hi <= 15) || fabsf(g.zero) > 4194304.f;
+  tg.clamp = !(c_lo >= 0 && c_hi <= 15) || fabsf(tg.zero) > 4194304.f;
   return tg;
 }
 
