@@ -126,21 +126,35 @@ __device__ __forceinline__ SignPlan make_plan(const TcParams& p) {
   return sp;
 }
 
-// bf16 bit pattern of A[m][k] (m = TMEM lane / output row, k = K index).
+// A[m][8j .. 8j+7] as one 16-byte chunk of bf16 +/-1 (m = TMEM lane / output row, k = K index).
+// F = 28: m = 32 h' + a (a < 28), k = 4 c + h2, A = H_28[a][c] (-1)^popc(h' & h2) times the row
+// sign of the outlier plan, sigma H_28[a][c_k] (-1)^popc(h' & e_hi); rows a >= 28 and columns
+// c >= 28 are zero. Power of two: A = (-1)^popc(m & k) times sigma (-1)^popc(m & e_hi).
 template <bool kF28>
-__device__ __forceinline__ uint16_t a_entry(int m, int k, const SignPlan& sp, const H28Masks& h) {
-  int neg;
+__device__ __forceinline__ uint4 a_chunk(int m, int j, const SignPlan& sp, const H28Masks& h) {
+  uint32_t neg = 0;  // bit e: entry k = 8j + e is -1
   if (kF28) {
-    const int hp = m >> 5, a = m & 31, c = k >> 2, h2 = k & 3;
-    if (a >= 28 || c >= 28) return 0;
-    neg = static_cast<int>((h.row[a] >> c) & 1u) ^ (__popc(hp & h2) & 1);
-    if (sp.active) neg ^= static_cast<int>((h.row[a] >> sp.c_k) & 1u) ^ (__popc(hp & sp.e_hi) & 1);
+    const int hp = m >> 5, a = m & 31;
+    if (a >= 28 || j >= 14) return make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t row = h.row[a];
+    uint32_t s = 0;
+    if (sp.active) s = ((row >> sp.c_k) & 1u) ^ (__popc(hp & sp.e_hi) & 1) ^ (sp.sigma < 0.f ? 1u : 0u);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t c = 2 * j + (e >> 2), h2 = e & 3;
+      neg |= (((row >> c) & 1u) ^ (__popc(hp & h2) & 1) ^ s) << e;
+    }
   } else {
-    neg = __popc(m & k) & 1;
-    if (sp.active) neg ^= __popc(m & sp.e_hi) & 1;
+    uint32_t s = __popc(m & (8 * j)) & 1;
+    if (sp.active) s ^= (__popc(m & sp.e_hi) & 1) ^ (sp.sigma < 0.f ? 1u : 0u);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) neg |= ((__popc(m & e) & 1) ^ s) << e;
   }
-  if (sp.active && sp.sigma < 0.f) neg ^= 1;
-  return neg ? 0xBF80 : 0x3F80;  // -1 / +1
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = (0x3F80u | (((neg >> (2 * i)) & 1u) << 15)) | ((0x3F80u | (((neg >> (2 * i + 1)) & 1u) << 15)) << 16);
+  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // K-major 128B-swizzled placement of A[m][k] (8-row x 64-element atoms, K halves 16 KB apart).
@@ -535,9 +549,9 @@ __global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_tc_kernel(const __
     fence_mbar_init();
   }
   // A = rowsign (.) (H_28 kron H_4) or rowsign (.) H_128, bf16, K-major SW128
-  for (int idx = threadIdx.x; idx < 128 * 128; idx += kThreads) {
-    const int m = idx >> 7, k = idx & 127;
-    *reinterpret_cast<uint16_t*>(a_smem + a_offset(m, k)) = a_entry<kF28>(m, k, sp, p.h);
+  for (int idx = threadIdx.x; idx < 128 * 16; idx += kThreads) {
+    const int m = idx >> 4, j = idx & 15;
+    *reinterpret_cast<uint4*>(a_smem + a_offset(m, 8 * j)) = a_chunk<kF28>(m, j, sp, p.h);
   }
   const int M = kF28 ? (1 << p.logM) : 0;
   // D as XOR masks on bf16 pairs, in the staged tile's (swizzled) order: 16-B chunk ch holds
@@ -906,9 +920,29 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
 
   const SignPlan sp = make_plan<kF28, kNcol>(p);
   const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
-  for (int idx = threadIdx.x; idx < 128 * 128; idx += kThreads) {
-    const int m = idx >> 7, k = idx & 127;
-    *reinterpret_cast<uint16_t*>(a_smem + a_offset(m, k)) = a_entry<kF28>(m, k, sp, p.h);
+  const int M = kF28 ? (1 << p.logM) : 0;
+  // D warps: their sign masks and tile destinations (global loads of D) ...
+  const bool last = per == kPerD;  // this warp also takes its lanes' kPerD-th chunk
+  uint4 mask[kPerD];
+  uint32_t dst[kPerD];
+  if (dwarp) {
+#pragma unroll
+    for (int u = 0; u < kPerD; ++u) {
+      const int L = (u < per ? c0 + 32 * u : c0) + lane;
+      const int k = L / (kNcol / 8), b0 = (L % (kNcol / 8)) * 8;
+      const int j0 = kF28 ? (k >> 2) * M + (k & 3) * kNcol + b0 : k * kNcol + b0;
+      mask[u] = chunk_sign_masks(*reinterpret_cast<const uint2*>(p.d + j0));  // 8 signs, 8-byte aligned
+      const int bp = b0 ^ static_cast<int>(col_xor & ~7u);  // where this chunk's columns go
+      const int nbp = bp >> 6, segp = (bp >> 3) & 7;
+      dst[u] = static_cast<uint32_t>(nbp) * kChunkBytes + k * 128 + ((segp ^ (k & 7)) << 4);
+    }
+  } else {
+    // ... while the other warps build A: rowsign (.) (H_28 kron H_4) or rowsign (.) H_128, K-major SW128
+    const int a_tid = threadIdx.x < kDWarp0 * 32 ? threadIdx.x : threadIdx.x - kDW * 32;
+    for (int idx = a_tid; idx < 128 * 16; idx += kThreads - kDW * 32) {
+      const int m = idx >> 4, j = idx & 15;
+      *reinterpret_cast<uint4*>(a_smem + a_offset(m, 8 * j)) = a_chunk<kF28>(m, j, sp, p.h);
+    }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -919,7 +953,6 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int M = kF28 ? (1 << p.logM) : 0;
 
   if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
@@ -950,19 +983,6 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
     }
   } else if (dwarp) {
     // ------------------------------------------------------------------ D pass: linear -> tile
-    const bool last = per == kPerD;  // this warp also takes its lanes' kPerD-th chunk
-    uint4 mask[kPerD];
-    uint32_t dst[kPerD];
-#pragma unroll
-    for (int u = 0; u < kPerD; ++u) {
-      const int L = (u < per ? c0 + 32 * u : c0) + lane;
-      const int k = L / (kNcol / 8), b0 = (L % (kNcol / 8)) * 8;
-      const int j0 = kF28 ? (k >> 2) * M + (k & 3) * kNcol + b0 : k * kNcol + b0;
-      mask[u] = chunk_sign_masks(*reinterpret_cast<const uint2*>(p.d + j0));  // 8 signs, 8-byte aligned
-      const int bp = b0 ^ static_cast<int>(col_xor & ~7u);  // where this chunk's columns go
-      const int nbp = bp >> 6, segp = (bp >> 3) & 7;
-      dst[u] = static_cast<uint32_t>(nbp) * kChunkBytes + k * 128 + ((segp ^ (k & 7)) << 4);
-    }
     int i = 0;
     for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
       const int st = i % S, bb = i % kTiles;
