@@ -57,9 +57,7 @@ using namespace ptx;
 // take alternate tokens (12 warps, 168 registers each: three warps share each SM sub-partition's
 // 16K-register file); at 256 columns a lane holds more values, so one group (8 warps, up to 255
 // registers). Each group's warp w reads TMEM lane quadrant w % 4.
-constexpr int kDWarps = 2;
 __host__ __device__ constexpr int epi_groups(int ncol) { return ncol <= 128 ? 2 : 1; }
-__host__ __device__ constexpr int threads_for(int ncol) { return 32 * (4 * epi_groups(ncol) + kDWarps + 2); }
 constexpr uint32_t kABytes = 128 * 128 * 2;  // A: 128 x 128 bf16
 constexpr uint32_t kBoxBytes = 16 * 128;     // one TMA box: 16 rows x 64 bf16 (128 B) = 2 KB
 constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23: fp32 whose ulp is 1
@@ -206,57 +204,12 @@ __device__ __forceinline__ void fwht_local(float2 (&p)[kPairs]) {
   if constexpr (kBits > 6) fwht_stage<kPairs, 6>(p);
 }
 
-// The D pass's column permutation within one 16-byte segment: element m moves to m ^ kF
-// (words by kF >> 1, the two bf16 halves of each word by kF & 1).
-template <int kF>
-__device__ __forceinline__ uint4 permute_segment(uint4 v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t o[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t t = w[i ^ (kF >> 1)];
-    o[i] = (kF & 1) ? __byte_perm(t, 0, 0x1032) : t;
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
-// One stage of the D pass: apply D's sign masks to every 16-byte chunk and move it to the slot
-// (chunk ^ seg_xor) of the same 128-byte row, permuting its 8 columns by kF.
-template <int kF, int kStageChunks, int kDThreads>
-__device__ __forceinline__ void d_pass_stage(uint4* base, const uint4* masks, int td, uint32_t seg_xor) {
-#pragma unroll 2
-  for (int c0 = 0; c0 < kStageChunks; c0 += 4 * kDThreads) {
-    uint4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int ch = c0 + u * kDThreads + td;
-      if (ch < kStageChunks) {
-        v[u] = base[ch];
-        const uint4 m = masks[ch];
-        v[u].x ^= m.x;
-        v[u].y ^= m.y;
-        v[u].z ^= m.z;
-        v[u].w ^= m.w;
-      }
-    }
-    __syncwarp();  // a row's 8 chunks are read by 8 lanes of this warp before any is rewritten
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int ch = c0 + u * kDThreads + td;
-      if (ch < kStageChunks) base[ch ^ static_cast<int>(seg_xor)] = permute_segment<kF>(v[u]);
-    }
-    __syncwarp();
-  }
-}
-
-// D's signs of one 16-byte chunk (8 bf16 columns) as XOR masks on its four 32-bit words.
-__device__ __forceinline__ uint4 chunk_sign_masks(uint2 d8) {
+// D's signs of one 16-byte chunk (8 bf16 columns, D at d8[0..8)) as XOR masks on its four
+// 32-bit words.
+__device__ __forceinline__ uint4 chunk_sign_masks(const int8_t* d8) {
   uint32_t w[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t pair = ((i < 2 ? d8.x : d8.y) >> (16 * (i & 1))) & 0xffffu;  // d[2i], d[2i+1]
-    w[i] = ((pair & 0x80u) << 8) | ((pair & 0x8000u) << 16);
-  }
+  for (int i = 0; i < 4; ++i) w[i] = (d8[2 * i] < 0 ? 0x8000u : 0u) | (d8[2 * i + 1] < 0 ? 0x80000000u : 0u);
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
@@ -308,20 +261,6 @@ __device__ __forceinline__ void tmem_load_pairs(uint32_t taddr, float2 (&p)[kPai
   }
 }
 
-template <int kPairs>
-__device__ __forceinline__ void tmem_store_pairs(uint32_t taddr, const float2 (&p)[kPairs]) {
-#pragma unroll
-  for (int c = 0; c < kPairs; c += 16) {
-    uint32_t r[32];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      r[2 * i] = __float_as_uint(p[c + i].x);
-      r[2 * i + 1] = __float_as_uint(p[c + i].y);
-    }
-    tmem_st32(taddr + 2 * c, r);
-  }
-  tmem_wait_st();
-}
 
 // Elementwise general sign vector: bit r of sbits flips the sign of column r.
 template <int kPairs>
@@ -365,23 +304,6 @@ __device__ __forceinline__ void local_minmax_xy(const float2 (&p)[kPairs], float
   lx = l0; hx = h0; ly = l1; hy = h1;
 }
 
-template <int kPairs>
-__device__ __forceinline__ void local_minmax(const float2 (&p)[kPairs], float& lo, float& hi) {
-  float l0 = p[0].x, l1 = p[0].y, h0 = p[0].x, h1 = p[0].y;
-#pragma unroll
-  for (int i = 1; i + 1 < kPairs; i += 2) {
-    l0 = fmin3(l0, p[i].x, p[i].y);
-    h0 = fmax3(h0, p[i].x, p[i].y);
-    l1 = fmin3(l1, p[i + 1].x, p[i + 1].y);
-    h1 = fmax3(h1, p[i + 1].x, p[i + 1].y);
-  }
-  if ((kPairs & 1) == 0) {
-    l0 = fmin3(l0, p[kPairs - 1].x, p[kPairs - 1].y);
-    h0 = fmax3(h0, p[kPairs - 1].x, p[kPairs - 1].y);
-  }
-  lo = fminf(lo, fminf(l0, l1));
-  hi = fmaxf(hi, fmaxf(h0, h1));
-}
 
 // Eight consecutive codes -> one u32 of nibbles (element 2i low nibble). u holds the bit
 // patterns of fma(w, c, zero + 1.5*2^23), whose low byte is the code (0..15).
@@ -485,334 +407,6 @@ __device__ __forceinline__ TokenGrid token_grid(float lo_w, float hi_w, float rs
 }
 
 // ------------------------------------------------------------------------------------- kernel
-
-template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
-__global__ void __launch_bounds__(threads_for(kNcol), 1) rotq_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcParams p) {
-  constexpr int kKRows = kF28 ? 112 : 128;     // K of the MMA chain
-  constexpr int kKSteps = kKRows / 16;
-  constexpr int kChunksN = kNcol / 64;          // 64-column TMA / swizzle atoms per token
-  constexpr int kBoxesPerChunk = kKRows / 16;
-  constexpr uint32_t kChunkBytes = kKRows * 128;
-  constexpr uint32_t kStageBytes = kChunksN * kChunkBytes;
-  constexpr uint32_t kTmemCols = 2 * kNcol < 32 ? 32 : 2 * kNcol;
-  constexpr int kPairs = kNcol <= 128 ? kNcol / 2 : 64;  // register pairs held per pass
-  constexpr int kStageChunks = kChunksN * kKRows * 8;  // 16-B chunks per stage
-  constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
-                              (static_cast<uint32_t>(kNcol >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
-  constexpr int kGroups = epi_groups(kNcol);
-  constexpr int kEpiWarps = 4 * kGroups;  // warps [0, kEpiWarps): epilogue
-  constexpr int kTmaWarp = kEpiWarps + kDWarps;  // then the D-pass warps, TMA, MMA
-  constexpr int kMmaWarp = kTmaWarp + 1;
-  constexpr int kThreads = threads_for(kNcol);
-  constexpr int kTBufs = 2 * kGroups;  // TMEM accumulators in flight
-  static_assert(kTBufs * kNcol <= 512, "TMEM holds 512 columns");
-
-  extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned base for the 128-byte swizzle atoms; offsetting the pointer (not casting
-  // through an integer) keeps the compiler's knowledge that every access below is to shared memory
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const int S = p.stages;
-  uint8_t* a_smem = smem;
-  uint32_t* dmask = reinterpret_cast<uint32_t*>(smem + kABytes);  // D sign masks, stage layout
-  uint8_t* ring = smem + kABytes + kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + S * kStageBytes);
-  uint64_t* full = bars;
-  uint64_t* dready = bars + S;
-  uint64_t* empty = bars + 2 * S;
-  uint64_t* tfull = bars + 3 * S;
-  uint64_t* tempty = bars + 3 * S + kTBufs;
-  uint64_t* redbar = bars + 3 * S + 2 * kTBufs;  // a group's min/max exchange, per TMEM buffer
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 3 * kTBufs);
-  float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [buffer][4 quadrants][lo, hi]
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const SignPlan sp = make_plan<kF28, kNcol>(p);
-  // The outlier-channel sign's column factor (-1)^popcount(b & e_lo) is applied as a column
-  // permutation of the MMA's input (diag(h_e) H = H P_e, P_e: b -> b ^ e): TMEM column b then
-  // holds input column b ^ e_lo. Bits >= 6 pick the 64-column TMA box, bits 3-5 the 16-byte
-  // slot the D pass writes, bits 0-2 the D pass's in-segment register permutation.
-  const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
-  const uint32_t seg_xor = (col_xor >> 3) & 7u;
-  const int box_xor = static_cast<int>(col_xor >> 6);
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) {
-      mbar_init(smem_u32(&full[i]), 1);
-      mbar_init(smem_u32(&dready[i]), kDWarps);
-      mbar_init(smem_u32(&empty[i]), 1);
-    }
-    for (int i = 0; i < kTBufs; ++i) {
-      mbar_init(smem_u32(&tfull[i]), 1);
-      mbar_init(smem_u32(&tempty[i]), 4);  // the 4 warps of the group that owns buffer i
-      mbar_init(smem_u32(&redbar[i]), 4);
-    }
-    fence_mbar_init();
-  }
-  // A = rowsign (.) (H_28 kron H_4) or rowsign (.) H_128, bf16, K-major SW128
-  for (int idx = threadIdx.x; idx < 128 * 16; idx += kThreads) {
-    const int m = idx >> 4, j = idx & 15;
-    *reinterpret_cast<uint4*>(a_smem + a_offset(m, 8 * j)) = a_chunk<kF28>(m, j, sp, p.h);
-  }
-  const int M = kF28 ? (1 << p.logM) : 0;
-  // D as XOR masks on bf16 pairs, in the staged tile's (swizzled) order: 16-B chunk ch holds
-  // row (K index) ch % (kKRows * 8) / 8, logical 8-column segment (slot ^ row) & 7
-  for (int ch = threadIdx.x; ch < kStageChunks; ch += kThreads) {
-    const int nb = ch / (kKRows * 8), rem = ch % (kKRows * 8);
-    const int row = rem >> 3, slot = rem & 7;
-    const int b0 = (nb ^ box_xor) * 64 + ((slot ^ (row & 7)) << 3);
-    const int j0 = kF28 ? (row >> 2) * M + (row & 3) * kNcol + b0 : row * kNcol + b0;
-#pragma unroll
-    for (int w = 0; w < 4; ++w)
-      dmask[4 * ch + w] = (p.d[j0 + 2 * w] < 0 ? 0x8000u : 0u) | (p.d[j0 + 2 * w + 1] < 0 ? 0x80000000u : 0u);
-  }
-  if (warp == kMmaWarp) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish();
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  if (warp == kTmaWarp) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&tmap);
-      int i = 0;
-      for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
-        const int st = i % S;
-        if (!mbar_wait(smem_u32(&empty[st]), ((i / S) & 1) ^ 1)) { flag_error(); break; }
-        const uint32_t fb = smem_u32(&full[st]);
-        mbar_arrive_expect_tx(fb, kStageBytes);
-        const uint32_t dst0 = smem_u32(ring + st * kStageBytes);
-#pragma unroll 1
-        for (int nb = 0; nb < kChunksN; ++nb) {
-#pragma unroll 1
-          for (int bx = 0; bx < kBoxesPerChunk; ++bx) {
-            const uint32_t dst = dst0 + nb * kChunkBytes + bx * kBoxBytes;
-            if (kF28)
-              tma_load_4d(dst, &tmap, (nb ^ box_xor) * 64, 0, bx * 4, t, fb);
-            else
-              tma_load_3d(dst, &tmap, (nb ^ box_xor) * 64, bx * 16, t, fb);
-          }
-        }
-      }
-      // do not leave the CTA with copies in flight: wait (bounded) for the last stages issued
-      const int issued = i;
-      for (int j = issued - S > 0 ? issued - S : 0; j < issued; ++j)
-        if (!mbar_wait(smem_u32(&full[j % S]), (j / S) & 1)) { flag_error(); break; }
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t a_base = smem_u32(a_smem);
-      int i = 0;
-      for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
-        const int st = i % S, tb = i % kTBufs;
-        if (!mbar_wait(smem_u32(&dready[st]), (i / S) & 1)) { flag_error(); break; }
-        if (!mbar_wait(smem_u32(&tempty[tb]), ((i / kTBufs) & 1) ^ 1)) { flag_error(); break; }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + tb * kNcol;
-        const uint32_t b_base = smem_u32(ring + st * kStageBytes);
-#pragma unroll
-        for (int ks = 0; ks < kKSteps; ++ks) {
-          const uint64_t ad = smem_desc(a_base + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc(b_base + ks * 2048, kChunkBytes, 1024);
-          mma_bf16(d_tmem, ad, bd, kIdesc, ks > 0 ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&empty[st]));
-        mma_commit(smem_u32(&tfull[tb]));
-      }
-      // leave no MMA in flight behind: the last commit must have landed before TMEM is freed
-      if (i > 0 && !mbar_wait(smem_u32(&tfull[(i - 1) % kTBufs]), ((i - 1) / kTBufs) & 1)) flag_error();
-    }
-  } else if (warp >= kEpiWarps) {
-    // ------------------------------------------------------------------ D pass (2 warps)
-    const int td = threadIdx.x - kEpiWarps * 32;
-    const uint4* masks = reinterpret_cast<const uint4*>(dmask);
-    int i = 0;
-    for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
-      const int st = i % S;
-      if (!mbar_wait(smem_u32(&full[st]), (i / S) & 1)) { flag_error(); break; }
-      uint4* base = reinterpret_cast<uint4*>(ring + st * kStageBytes);
-      constexpr int kDT = kDWarps * 32;
-      switch (col_xor & 7u) {  // low three bits of the column permutation, fixed per launch
-        case 0: d_pass_stage<0, kStageChunks, kDT>(base, masks, td, seg_xor); break;
-        case 1: d_pass_stage<1, kStageChunks, kDT>(base, masks, td, seg_xor); break;
-        case 2: d_pass_stage<2, kStageChunks, kDT>(base, masks, td, seg_xor); break;
-        case 3: d_pass_stage<3, kStageChunks, kDT>(base, masks, td, seg_xor); break;
-        case 4: d_pass_stage<4, kStageChunks, kDT>(base, masks, td, seg_xor); break;
-        case 5: d_pass_stage<5, kStageChunks, kDT>(base, masks, td, seg_xor); break;
-        case 6: d_pass_stage<6, kStageChunks, kDT>(base, masks, td, seg_xor); break;
-        default: d_pass_stage<7, kStageChunks, kDT>(base, masks, td, seg_xor); break;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&dready[st]));
-    }
-  } else {
-    // ------------------------------------------------------------------ epilogue
-    const int quad = warp & 3, group = warp >> 2;
-    const bool active = !kF28 || lane < 28;
-    // this lane's output run: row (h2' = quad, a = lane) or r = quad * 32 + lane
-    const int64_t j0 = kF28 ? static_cast<int64_t>(lane) * M + quad * kNcol : static_cast<int64_t>(quad * 32 + lane) * kNcol;
-    uint32_t sbits[kVecSign ? kNcol / 32 : 1];
-    if (kVecSign) {
-#pragma unroll
-      for (int w = 0; w < kNcol / 32; ++w) {
-        uint32_t b = 0;
-        if (active)
-          for (int r = 0; r < 32; ++r) b |= (p.s[j0 + 32 * w + r] < 0 ? 1u : 0u) << r;
-        sbits[w] = b;
-      }
-    }
-    const float rs = p.inv_sqrt_n;
-    // this group takes every kGroups-th of the CTA's tokens, starting at its index
-    int i = group;
-    for (int t = blockIdx.x + group * gridDim.x; t < p.T; t += kGroups * gridDim.x, i += kGroups) {
-      const int tb = i % kTBufs;
-      if (!mbar_wait(smem_u32(&tfull[tb]), (i / kTBufs) & 1)) { flag_error(); break; }
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tb * kNcol;
-      float2 v[kPairs];
-      float lo = pos_inf(), hi = -pos_inf();
-      if constexpr (kNcol <= 128) {
-        tmem_load_pairs<0, kPairs>(taddr, v);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&tempty[tb]));
-        fwht_local<kPairs, (kNcol == 64 ? 6 : 7)>(v);
-        if (kVecSign) apply_sign_bits<kPairs>(v, sbits);
-        if (active) local_minmax<kPairs>(v, lo, hi);
-      } else {
-        // 256 columns: two 128-column halves through the registers, then the top stage
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          tmem_load_pairs<0, kPairs>(taddr + hh * 128, v);
-          fwht_local<kPairs, 7>(v);
-          tmem_store_pairs<kPairs>(taddr + hh * 128, v);
-        }
-#pragma unroll 1
-        for (int g = 0; g < 2; ++g) {
-          float2 u[32];
-          tmem_load_pairs<0, 32>(taddr + g * 64, v);
-          tmem_load_pairs<0, 32>(taddr + 128 + g * 64, u);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const float2 a = v[k], b = u[k];
-            v[k] = __fadd2_rn(a, b);
-            v[32 + k] = fsub2(a, b);
-          }
-          if (kVecSign) {
-            const uint32_t sb[2] = {sbits[2 * g], sbits[2 * g + 1]};
-            const uint32_t sb2[2] = {sbits[4 + 2 * g], sbits[4 + 2 * g + 1]};
-            float2 lo_half[32], hi_half[32];
-#pragma unroll
-            for (int k = 0; k < 32; ++k) { lo_half[k] = v[k]; hi_half[k] = v[32 + k]; }
-            apply_sign_bits<32>(lo_half, sb);
-            apply_sign_bits<32>(hi_half, sb2);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) { v[k] = lo_half[k]; v[32 + k] = hi_half[k]; }
-          }
-          if (active) local_minmax<64>(v, lo, hi);
-        }
-      }
-      // token min/max: warp, then the 4 epilogue warps through shared memory
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-      }
-      if (lane == 0) {
-        red[(tb * 4 + quad) * 2] = lo;
-        red[(tb * 4 + quad) * 2 + 1] = hi;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&redbar[tb]));
-      if (!mbar_wait(smem_u32(&redbar[tb]), (i / kTBufs) & 1)) { flag_error(); break; }
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        lo = fminf(lo, red[(tb * 4 + w) * 2]);
-        hi = fmaxf(hi, red[(tb * 4 + w) * 2 + 1]);
-      }
-      if (kQuant) {
-        const TokenGrid g = token_grid(lo, hi, rs, p.clip);
-        if (quad == 0 && lane == 0) {
-          p.scale[t] = g.scale;
-          p.zero[t] = g.zero;
-        }
-        uint8_t* qrow = p.q + static_cast<int64_t>(t) * (p.n >> 1);
-        if constexpr (kNcol <= 128) {
-          if (active) quant_store<kPairs>(v, make_float2(g.c, g.c), g.zm, g.clamp, qrow + (j0 >> 1));
-        } else {
-#pragma unroll 1
-          for (int gg = 0; gg < 2; ++gg) {
-            float2 u[32], lo_half[32], hi_half[32];
-            tmem_load_pairs<0, 32>(taddr + gg * 64, lo_half);
-            tmem_load_pairs<0, 32>(taddr + 128 + gg * 64, u);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              const float2 a = lo_half[k], b = u[k];
-              lo_half[k] = __fadd2_rn(a, b);
-              hi_half[k] = fsub2(a, b);
-            }
-            if (kVecSign) {
-              const uint32_t sb[2] = {sbits[2 * gg], sbits[2 * gg + 1]};
-              const uint32_t sb2[2] = {sbits[4 + 2 * gg], sbits[4 + 2 * gg + 1]};
-              apply_sign_bits<32>(lo_half, sb);
-              apply_sign_bits<32>(hi_half, sb2);
-            }
-            if (active) {
-              quant_store<32>(lo_half, make_float2(g.c, g.c), g.zm, g.clamp, qrow + ((j0 + gg * 64) >> 1));
-              quant_store<32>(hi_half, make_float2(g.c, g.c), g.zm, g.clamp, qrow + ((j0 + 128 + gg * 64) >> 1));
-            }
-          }
-        }
-      } else {
-        float* yrow = p.y + static_cast<int64_t>(t) * p.ldy;
-        if constexpr (kNcol <= 128) {
-          if (active) store_y<kPairs>(v, rs, yrow + j0);
-        } else {
-#pragma unroll 1
-          for (int gg = 0; gg < 2; ++gg) {
-            float2 u[32], lo_half[32], hi_half[32];
-            tmem_load_pairs<0, 32>(taddr + gg * 64, lo_half);
-            tmem_load_pairs<0, 32>(taddr + 128 + gg * 64, u);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              const float2 a = lo_half[k], b = u[k];
-              lo_half[k] = __fadd2_rn(a, b);
-              hi_half[k] = fsub2(a, b);
-            }
-            if (kVecSign) {
-              const uint32_t sb[2] = {sbits[2 * gg], sbits[2 * gg + 1]};
-              const uint32_t sb2[2] = {sbits[4 + 2 * gg], sbits[4 + 2 * gg + 1]};
-              apply_sign_bits<32>(lo_half, sb);
-              apply_sign_bits<32>(hi_half, sb2);
-            }
-            if (active) {
-              store_y<32>(lo_half, rs, yrow + j0 + gg * 64);
-              store_y<32>(hi_half, rs, yrow + j0 + 128 + gg * 64);
-            }
-          }
-        }
-      }
-      if constexpr (kNcol > 128) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&tempty[tb]));
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == kMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
-  }
-}
 
 // ------------------------------------------------------------- streamed variant (<= 128 columns)
 //
@@ -931,7 +525,7 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
       const int L = (u < per ? c0 + 32 * u : c0) + lane;
       const int k = L / (kNcol / 8), b0 = (L % (kNcol / 8)) * 8;
       const int j0 = kF28 ? (k >> 2) * M + (k & 3) * kNcol + b0 : k * kNcol + b0;
-      mask[u] = chunk_sign_masks(*reinterpret_cast<const uint2*>(p.d + j0));  // 8 signs, 8-byte aligned
+      mask[u] = chunk_sign_masks(p.d + j0);
       const int bp = b0 ^ static_cast<int>(col_xor & ~7u);  // where this chunk's columns go
       const int nbp = bp >> 6, segp = (bp >> 3) & 7;
       dst[u] = static_cast<uint32_t>(nbp) * kChunkBytes + k * 128 + ((segp ^ (k & 7)) << 4);
@@ -1101,6 +695,315 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
   }
 }
 
+// ------------------------------------------------------------------ 256 columns: half-row epilogue
+//
+// A 256-column row per token is 56-64 KB, so the input is staged by tensor-map TMA boxes straight
+// into the swizzled MMA tile (three stages fit beside A), and two D warps convert each stage in
+// place: sign flips, the word permutation, and the permutation of the 16-byte slots inside each
+// 128-byte row (column bits 3-5; bits 6-7 pick the TMA box, bit 0 is folded into the epilogue).
+// One N = 256 MMA chain per token writes Z = [Z0 | Z1] (input columns 0..127 | 128..255) to TMEM.
+// Eight epilogue warps share a token: the warp for half h and lane quadrant q forms
+// Y_h = Z0 + (-1)^h Z1 -- the column butterfly on bit 7 -- 16 columns at a time, then runs the
+// remaining seven butterfly stages, min/max, the 8-warp exchange and quantization on its 128
+// values.
+
+constexpr int kWideEpiWarps = 8;
+constexpr int kWideDWarps = 2;
+constexpr int kWideThreads = 32 * (kWideEpiWarps + kWideDWarps + 2);
+constexpr int kWideTBufs = 2;
+
+// One stage of the in-place D pass (packed sign words, see chunk_sign_bits): chunk ch is read,
+// its signs flipped and words moved by kW, and written to slot ch ^ seg_xor of the same 128-byte
+// row. A row's 8 chunks belong to 8 lanes of one warp and one batch, read before any is written.
+template <int kW, int kPerD, int kDT, int kBatch>
+__device__ __forceinline__ void inplace_d_pass_bits(uint4* base, const uint32_t (&bits_in)[kPerD], int td,
+                                                    uint32_t seg_xor) {
+  uint32_t bits[kPerD];
+#pragma unroll
+  for (int u = 0; u < kPerD; ++u) {
+    bits[u] = bits_in[u];
+    asm volatile("" : "+r"(bits[u]));
+  }
+#pragma unroll
+  for (int u0 = 0; u0 < kPerD; u0 += kBatch) {
+    uint4 v[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b)
+      if (u0 + b < kPerD) v[b] = base[(u0 + b) * kDT + td];
+    __syncwarp();
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      if (u0 + b < kPerD) {
+        const uint32_t m = bits[u0 + b];
+        const uint32_t w[4] = {v[b].x ^ (m & 0x80008000u), v[b].y ^ ((m << 1) & 0x80008000u),
+                               v[b].z ^ ((m << 2) & 0x80008000u), v[b].w ^ ((m << 3) & 0x80008000u)};
+        base[((u0 + b) * kDT + td) ^ static_cast<int>(seg_xor)] = make_uint4(w[kW], w[1 ^ kW], w[2 ^ kW], w[3 ^ kW]);
+      }
+    }
+    __syncwarp();
+  }
+}
+
+template <bool kF28, bool kVecSign, bool kQuant>
+__global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                                    TcParams p) {
+  constexpr int kNcol = 256, kHalf = 128, kPairs = 64;
+  constexpr int kKRows = kF28 ? 112 : 128;
+  constexpr int kKSteps = kKRows / 16;
+  constexpr int kChunksN = kNcol / 64;
+  constexpr int kBoxesPerChunk = kKRows / 16;
+  constexpr uint32_t kChunkBytes = kKRows * 128;
+  constexpr uint32_t kStageBytes = kChunksN * kChunkBytes;
+  constexpr int kStageChunks = static_cast<int>(kStageBytes / 16);
+  constexpr int kDT = kWideDWarps * 32;
+  constexpr int kPerD = kStageChunks / kDT;
+  static_assert(kStageChunks % kDT == 0, "D lanes own whole chunks");
+  constexpr int kDBatch = 4;
+  constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                              (static_cast<uint32_t>(kNcol >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+  constexpr int kDWarp0 = kWideEpiWarps;
+  constexpr int kTmaWarp = kDWarp0 + kWideDWarps;
+  constexpr int kMmaWarp = kTmaWarp + 1;
+  constexpr int kThreads = kWideThreads;
+  constexpr int kTBufs = kWideTBufs;
+  constexpr uint32_t kTmemCols = kTBufs * kNcol;
+  static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int S = p.stages;
+  uint8_t* a_smem = smem;
+  uint8_t* ring = smem + kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + S * kStageBytes);
+  uint64_t* full = bars;
+  uint64_t* dready = bars + S;
+  uint64_t* empty = bars + 2 * S;
+  uint64_t* tfull = bars + 3 * S;
+  uint64_t* tempty = tfull + kTBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + kTBufs);
+  float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [token parity][half][quadrant][lo, hi]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const SignPlan sp = make_plan<kF28, kNcol>(p);
+  const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
+  const uint32_t seg_xor = (col_xor >> 3) & 7u;
+  const int box_xor = static_cast<int>(col_xor >> 6);
+  const int M = kF28 ? (1 << p.logM) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&dready[i]), kWideDWarps);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    for (int i = 0; i < kTBufs; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), kWideEpiWarps);
+    }
+    fence_mbar_init();
+  }
+  const bool dwarp = warp >= kDWarp0 && warp < kTmaWarp;
+  const int td = threadIdx.x - kDWarp0 * 32;
+  uint32_t bits[kPerD];
+  if (dwarp) {
+    // D signs of this lane's chunks, in the staged tile's order: chunk ch holds row (K index)
+    // ch % (kKRows * 8) / 8, input columns of box (nb ^ box_xor), segment (slot ^ row) & 7
+#pragma unroll
+    for (int u = 0; u < kPerD; ++u) {
+      const int ch = u * kDT + td;
+      const int nb = ch / (kKRows * 8), rem = ch % (kKRows * 8);
+      const int row = rem >> 3, slot = rem & 7;
+      const int b0 = (nb ^ box_xor) * 64 + ((slot ^ (row & 7)) << 3);
+      const int j0 = kF28 ? (row >> 2) * M + (row & 3) * kNcol + b0 : row * kNcol + b0;
+      uint32_t b = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) b |= (p.d[j0 + e] < 0 ? 1u : 0u) << (15 + 16 * (e & 1) - (e >> 1));
+      bits[u] = b;
+    }
+  } else {
+    const int a_tid = threadIdx.x < kDWarp0 * 32 ? threadIdx.x : threadIdx.x - kWideDWarps * 32;
+    for (int idx = a_tid; idx < 128 * 16; idx += kThreads - kWideDWarps * 32) {
+      const int m = idx >> 4, j = idx & 15;
+      *reinterpret_cast<uint4*>(a_smem + a_offset(m, 8 * j)) = a_chunk<kF28>(m, j, sp, p.h);
+    }
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmap);
+      int i = 0;
+      for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+        const int st = i % S;
+        if (!mbar_wait(smem_u32(&empty[st]), ((i / S) & 1) ^ 1)) { flag_error(); break; }
+        const uint32_t fb = smem_u32(&full[st]);
+        mbar_arrive_expect_tx(fb, kStageBytes);
+        const uint32_t dst0 = smem_u32(ring + st * kStageBytes);
+#pragma unroll 1
+        for (int nb = 0; nb < kChunksN; ++nb) {
+#pragma unroll 1
+          for (int bx = 0; bx < kBoxesPerChunk; ++bx) {
+            const uint32_t dst = dst0 + nb * kChunkBytes + bx * kBoxBytes;
+            if (kF28)
+              tma_load_4d(dst, &tmap, (nb ^ box_xor) * 64, 0, bx * 4, t, fb);
+            else
+              tma_load_3d(dst, &tmap, (nb ^ box_xor) * 64, bx * 16, t, fb);
+          }
+        }
+      }
+      // do not leave the CTA with copies in flight: wait (bounded) for the last stages issued
+      const int issued = i;
+      for (int j = issued - S > 0 ? issued - S : 0; j < issued; ++j)
+        if (!mbar_wait(smem_u32(&full[j % S]), (j / S) & 1)) { flag_error(); break; }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t a_base = smem_u32(a_smem);
+      int i = 0;
+      for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+        const int st = i % S, tb = i % kTBufs;
+        if (!mbar_wait(smem_u32(&dready[st]), (i / S) & 1) ||
+            !mbar_wait(smem_u32(&tempty[tb]), ((i / kTBufs) & 1) ^ 1)) {
+          flag_error();
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + tb * kNcol;
+        const uint32_t b_base = smem_u32(ring + st * kStageBytes);
+#pragma unroll
+        for (int ks = 0; ks < kKSteps; ++ks) {
+          const uint64_t ad = smem_desc(a_base + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc(b_base + ks * 2048, kChunkBytes, 1024);
+          mma_bf16(d_tmem, ad, bd, kIdesc, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&empty[st]));
+        mma_commit(smem_u32(&tfull[tb]));
+      }
+      if (i > 0 && !mbar_wait(smem_u32(&tfull[(i - 1) % kTBufs]), ((i - 1) / kTBufs) & 1)) flag_error();
+    }
+  } else if (dwarp) {
+    // ------------------------------------------------------------------ D pass, in place
+    int i = 0;
+    for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+      const int st = i % S;
+      if (!warp_wait(smem_u32(&full[st]), (i / S) & 1)) { flag_error(); break; }
+      uint4* base = reinterpret_cast<uint4*>(ring + st * kStageBytes);
+      switch ((col_xor >> 1) & 3u) {
+        case 0: inplace_d_pass_bits<0, kPerD, kDT, kDBatch>(base, bits, td, seg_xor); break;
+        case 1: inplace_d_pass_bits<1, kPerD, kDT, kDBatch>(base, bits, td, seg_xor); break;
+        case 2: inplace_d_pass_bits<2, kPerD, kDT, kDBatch>(base, bits, td, seg_xor); break;
+        default: inplace_d_pass_bits<3, kPerD, kDT, kDBatch>(base, bits, td, seg_xor); break;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&dready[st]));
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue: one half row per thread
+    const int quad = warp & 3, half = warp >> 2;
+    const bool active = !kF28 || lane < 28;
+    const int64_t j0 = (kF28 ? static_cast<int64_t>(lane) * M + quad * kNcol
+                             : static_cast<int64_t>(quad * 32 + lane) * kNcol) + half * kHalf;
+    uint32_t sbits[kVecSign ? kHalf / 32 : 1];
+    if (kVecSign) {
+#pragma unroll
+      for (int w = 0; w < kHalf / 32; ++w) {
+        uint32_t b = 0;
+        if (active)
+          for (int r = 0; r < 32; ++r) b |= (p.s[j0 + 32 * w + r] < 0 ? 1u : 0u) << r;
+        sbits[w] = b;
+      }
+    }
+    const float rs = p.inv_sqrt_n;
+    const bool odd_neg = (col_xor & 1u) != 0;  // see rotq_stream_kernel
+    bool live = true;
+    int i = 0;
+    for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+      const int tb = i % kTBufs;
+      if (live && !warp_wait(smem_u32(&tfull[tb]), (i / kTBufs) & 1)) {
+        flag_error();
+        live = false;
+      }
+      if (!live) {
+        named_barrier_sync(1, 32 * kWideEpiWarps);
+        continue;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tb * kNcol;
+      // Y_h = Z0 + (-1)^h Z1, sixteen columns at a time. When the outlier permutation swaps the
+      // halves (bit 7) this gives Z1 + Z0 and Z1 - Z0 = -(Z0 - Z1): bit for bit the sign-adjusted
+      // values, as with the other permutation bits.
+      float2 v[kPairs];
+#pragma unroll
+      for (int c = 0; c < kHalf; c += 16) {
+        uint32_t r1[16];
+        tmem_ld16_pair(taddr + c, taddr + kHalf + c, v + c / 2, r1);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float2 z1 = make_float2(__uint_as_float(r1[2 * k]), __uint_as_float(r1[2 * k + 1]));
+          v[c / 2 + k] = half ? fsub2(v[c / 2 + k], z1) : __fadd2_rn(v[c / 2 + k], z1);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty[tb]));
+      fwht_local<kPairs, 7>(v);
+      if (kVecSign) apply_sign_bits<kPairs>(v, sbits);
+      float lo = pos_inf(), hi = -pos_inf();
+      if (active) {
+        float lx, hx, ly, hy;
+        local_minmax_xy<kPairs>(v, lx, hx, ly, hy);
+        lo = fminf(lx, odd_neg ? -hy : ly);
+        hi = fmaxf(hx, odd_neg ? -ly : hy);
+      }
+      lo = warp_min(lo);
+      hi = warp_max(hi);
+      // exchange slots alternate per token: a slot is rewritten only after the next token's
+      // barrier, which every epilogue warp passes after reading it
+      float* rslot = red + (i & 1) * 16;
+      if (lane == 0) {
+        rslot[(half * 4 + quad) * 2] = lo;
+        rslot[(half * 4 + quad) * 2 + 1] = hi;
+      }
+      named_barrier_sync(1, 32 * kWideEpiWarps);  // the token's eight partial extremes are in
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        lo = fminf(lo, rslot[w * 2]);
+        hi = fmaxf(hi, rslot[w * 2 + 1]);
+      }
+      if (kQuant) {
+        const TokenGrid g = token_grid(lo, hi, rs, p.clip);
+        if (warp == 0 && lane == 0) {
+          p.scale[t] = g.scale;
+          p.zero[t] = g.zero;
+        }
+        if (active)
+          quant_store<kPairs>(v, make_float2(g.c, odd_neg ? -g.c : g.c), g.zm, g.clamp,
+                              p.q + static_cast<int64_t>(t) * (p.n >> 1) + (j0 >> 1));
+      } else if (active) {
+        store_y<kPairs>(v, rs, p.y + static_cast<int64_t>(t) * p.ldy + j0, odd_neg ? -rs : rs);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------------------------- host
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -1117,25 +1020,33 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
-cudaError_t launch_tc(const CUtensorMap& tmap, const TcParams& p0, cudaStream_t st) {
+template <bool kF28, bool kVecSign, bool kQuant>
+cudaError_t launch_wide(const CUtensorMap& tmap, const TcParams& p0, cudaStream_t st) {
   constexpr int kKRows = kF28 ? 112 : 128;
-  constexpr uint32_t kStageBytes = (kNcol / 64) * kKRows * 128;
-  constexpr uint32_t kSmemBudget = 227 * 1024 - 1024 - kABytes - kStageBytes - 512;
+  constexpr uint32_t kStageBytes = 4 * kKRows * 128;
+  constexpr uint32_t kSmemBudget = 227 * 1024 - 1024 - kABytes - 1024;
   TcParams p = p0;
   p.stages = static_cast<int>(kSmemBudget / kStageBytes);
   if (p.stages > 8) p.stages = 8;
-  const size_t smem = 1024 + kABytes + kStageBytes + static_cast<size_t>(p.stages) * kStageBytes + 512;
-  auto kern = rotq_tc_kernel<kNcol, kF28, kVecSign, kQuant>;
+  if (p.stages < 2) return cudaErrorNotSupported;
+  const size_t smem = 1024 + kABytes + static_cast<size_t>(p.stages) * kStageBytes + 1024;
+  auto kern = rotq_wide_kernel<kF28, kVecSign, kQuant>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int grid = p.T < sms ? p.T : sms;
-  kern<<<grid, threads_for(kNcol), smem, st>>>(tmap, p);
+  kern<<<grid, kWideThreads, smem, st>>>(tmap, p);
   count_launch();
   return cudaGetLastError();
+}
+
+template <bool kF28>
+cudaError_t dispatch_wide(const CUtensorMap& tmap, const TcParams& p, bool vec_sign, bool quant, cudaStream_t st) {
+  if (vec_sign)
+    return quant ? launch_wide<kF28, true, true>(tmap, p, st) : launch_wide<kF28, true, false>(tmap, p, st);
+  return quant ? launch_wide<kF28, false, true>(tmap, p, st) : launch_wide<kF28, false, false>(tmap, p, st);
 }
 
 template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
@@ -1165,13 +1076,6 @@ cudaError_t dispatch_stream(const TcParams& p, bool vec_sign, bool quant, cudaSt
   if (vec_sign)
     return quant ? launch_stream<kNcol, kF28, true, true>(p, st) : launch_stream<kNcol, kF28, true, false>(p, st);
   return quant ? launch_stream<kNcol, kF28, false, true>(p, st) : launch_stream<kNcol, kF28, false, false>(p, st);
-}
-
-template <int kNcol, bool kF28>
-cudaError_t dispatch_mode(const CUtensorMap& tmap, const TcParams& p, bool vec_sign, bool quant, cudaStream_t st) {
-  if (vec_sign)
-    return quant ? launch_tc<kNcol, kF28, true, true>(tmap, p, st) : launch_tc<kNcol, kF28, true, false>(tmap, p, st);
-  return quant ? launch_tc<kNcol, kF28, false, true>(tmap, p, st) : launch_tc<kNcol, kF28, false, false>(tmap, p, st);
 }
 
 }  // namespace
@@ -1204,12 +1108,9 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
   p.inv_sqrt_n = a.inv_sqrt_n;
   p.h = h;
   const bool vec = a.s != nullptr && a.kp == nullptr;
-  // Streamed variant for rows of up to 128 columns per token (D read 8 bytes at a time); 256-column
-  // rows, whose lane lines do not fit in registers at once, take the tensor-map kernel.
-  if (reinterpret_cast<uintptr_t>(a.d) % 8 == 0) {
-    if (ncol == 64) return f28 ? dispatch_stream<64, true>(p, vec, quant, st) : dispatch_stream<64, false>(p, vec, quant, st);
-    if (ncol == 128) return f28 ? dispatch_stream<128, true>(p, vec, quant, st) : dispatch_stream<128, false>(p, vec, quant, st);
-  }
+  // Up to 128 columns per token: the streamed kernel; 256 columns: the TMA-staged wide kernel.
+  if (ncol == 64) return f28 ? dispatch_stream<64, true>(p, vec, quant, st) : dispatch_stream<64, false>(p, vec, quant, st);
+  if (ncol == 128) return f28 ? dispatch_stream<128, true>(p, vec, quant, st) : dispatch_stream<128, false>(p, vec, quant, st);
 
   auto encode = encode_fn();
   if (encode == nullptr) return cudaErrorNotSupported;
@@ -1234,14 +1135,7 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   }
   if (r != CUDA_SUCCESS) return cudaErrorNotSupported;
-  if (f28) {
-    if (ncol == 64) return dispatch_mode<64, true>(tmap, p, vec, quant, st);
-    if (ncol == 128) return dispatch_mode<128, true>(tmap, p, vec, quant, st);
-    return dispatch_mode<256, true>(tmap, p, vec, quant, st);
-  }
-  if (ncol == 64) return dispatch_mode<64, false>(tmap, p, vec, quant, st);
-  if (ncol == 128) return dispatch_mode<128, false>(tmap, p, vec, quant, st);
-  return dispatch_mode<256, false>(tmap, p, vec, quant, st);
+  return f28 ? dispatch_wide<true>(tmap, p, vec, quant, st) : dispatch_wide<false>(tmap, p, vec, quant, st);
 }
 
 cudaError_t read_device_error(uint32_t* out, bool clear) {
