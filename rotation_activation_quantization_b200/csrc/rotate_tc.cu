@@ -90,26 +90,41 @@ struct TcParams {
 
 // Structured sign vector: sigma * g(a) * (-1)^popcount(hi & e_hi) * (-1)^popcount(b & e_lo).
 struct SignPlan {
-  float sigma;
   int32_t c_k;       // F = 28: H_28 column of the outlier (g(a) = H_28[a][c_k])
   uint32_t e_hi;     // bits of the outlier index that index A's rows (h2 or r)
   uint32_t e_lo;     // bits that index the TMEM columns: applied as the column permutation b ^ e_lo
   bool active;
 };
 
+// The outlier's index k and value x_k, loaded by every thread before anything else: plain loads
+// issued ahead of the CTA's first bulk copies, used only once those are on their way.
+struct OutlierRef {
+  int32_t k;
+  float xk;
+};
+__device__ __forceinline__ OutlierRef load_outlier(const TcParams& p) {
+  OutlierRef o{-1, 0.f};
+  if (p.kp != nullptr) {
+    o.k = *p.kp;
+    o.xk = *p.xkp;
+  }
+  return o;
+}
+
+// The parts of s = sigma * H[:, k] that do not depend on D: its column part e_lo, row part e_hi
+// and H_28 column c_k. sigma = sgn(x_k) sgn(D_k), a sign on every output, is applied by the
+// epilogue (outlier_sigma), which has time to load D_k.
 template <bool kF28, int kNcol>
-__device__ __forceinline__ SignPlan make_plan(const TcParams& p) {
-  SignPlan sp{1.f, 0, 0u, 0u, false};
+__device__ __forceinline__ SignPlan make_plan(const TcParams& p, OutlierRef o) {
+  SignPlan sp{0, 0u, 0u, false};
   if (p.kp == nullptr) return sp;
-  const int k = *p.kp;
-  const float xk = *p.xkp;
+  const int k = o.k;
   if (k < 0 || k >= p.n) {  // not a channel: report it and apply no sign adjustment
     flag_error(2u);
     return sp;
   }
-  if (xk == 0.f) return sp;  // s_j = sgn(+/-0) = +1 everywhere
+  if (o.xk == 0.f) return sp;  // s_j = sgn(+/-0) = +1 everywhere
   sp.active = true;
-  sp.sigma = ((xk < 0.f) != (p.d[k] < 0)) ? -1.f : 1.f;
   constexpr int kLogNcol = kNcol == 64 ? 6 : (kNcol == 128 ? 7 : 8);
   if (kF28) {
     const int M = 1 << p.logM;
@@ -124,10 +139,15 @@ __device__ __forceinline__ SignPlan make_plan(const TcParams& p) {
   return sp;
 }
 
+// True when sigma = sgn(x_k) sgn(D_k) is -1 for an active plan: every output changes sign.
+__device__ __forceinline__ bool outlier_sigma_neg(const TcParams& p, const SignPlan& sp, OutlierRef o) {
+  return sp.active && ((o.xk < 0.f) != (p.d[o.k] < 0));
+}
+
 // A[m][8j .. 8j+7] as one 16-byte chunk of bf16 +/-1 (m = TMEM lane / output row, k = K index).
 // F = 28: m = 32 h' + a (a < 28), k = 4 c + h2, A = H_28[a][c] (-1)^popc(h' & h2) times the row
-// sign of the outlier plan, sigma H_28[a][c_k] (-1)^popc(h' & e_hi); rows a >= 28 and columns
-// c >= 28 are zero. Power of two: A = (-1)^popc(m & k) times sigma (-1)^popc(m & e_hi).
+// sign of the outlier plan, H_28[a][c_k] (-1)^popc(h' & e_hi); rows a >= 28 and columns c >= 28
+// are zero. Power of two: A = (-1)^popc(m & k) times (-1)^popc(m & e_hi).
 template <bool kF28>
 __device__ __forceinline__ uint4 a_chunk(int m, int j, const SignPlan& sp, const H28Masks& h) {
   uint32_t neg = 0;  // bit e: entry k = 8j + e is -1
@@ -136,7 +156,7 @@ __device__ __forceinline__ uint4 a_chunk(int m, int j, const SignPlan& sp, const
     if (a >= 28 || j >= 14) return make_uint4(0u, 0u, 0u, 0u);
     const uint32_t row = h.row[a];
     uint32_t s = 0;
-    if (sp.active) s = ((row >> sp.c_k) & 1u) ^ (__popc(hp & sp.e_hi) & 1) ^ (sp.sigma < 0.f ? 1u : 0u);
+    if (sp.active) s = ((row >> sp.c_k) & 1u) ^ (__popc(hp & sp.e_hi) & 1);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const uint32_t c = 2 * j + (e >> 2), h2 = e & 3;
@@ -144,7 +164,7 @@ __device__ __forceinline__ uint4 a_chunk(int m, int j, const SignPlan& sp, const
     }
   } else {
     uint32_t s = __popc(m & (8 * j)) & 1;
-    if (sp.active) s ^= (__popc(m & sp.e_hi) & 1) ^ (sp.sigma < 0.f ? 1u : 0u);
+    if (sp.active) s ^= __popc(m & sp.e_hi) & 1;
 #pragma unroll
     for (int e = 0; e < 8; ++e) neg |= ((__popc(m & e) & 1) ^ s) << e;
   }
@@ -474,6 +494,7 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
   float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [buffer][4 quadrants][lo, hi]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const OutlierRef orf = load_outlier(p);  // issued ahead of the bulk copies
   if (threadIdx.x == 0) {
     for (int i = 0; i < S * kDW; ++i) mbar_init(smem_u32(&lfull[i]), 1);
     for (int i = 0; i < kTiles; ++i) {
@@ -512,7 +533,7 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
     }
   }
 
-  const SignPlan sp = make_plan<kF28, kNcol>(p);
+  const SignPlan sp = make_plan<kF28, kNcol>(p, orf);
   const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
   const int M = kF28 ? (1 << p.logM) : 0;
   // D warps: their sign masks and tile destinations (global loads of D) ...
@@ -629,6 +650,7 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
     const float rs = p.inv_sqrt_n;
     // the outlier permutation's bit 0 is not applied to the input: every odd column of the
     // transform comes out negated (H P_1 = diag((-1)^j) H), which min/max and quantization undo
+    const bool sneg = outlier_sigma_neg(p, sp, orf);  // every output negated
     const bool odd_neg = (col_xor & 1u) != 0;
     // A warp whose wait runs out stops working but keeps taking its group's barrier, once per token
     // like the others, so that no warp of the group is left waiting there.
@@ -672,6 +694,11 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
         lo = fminf(lo, red[(tb * 4 + w) * 2]);
         hi = fmaxf(hi, red[(tb * 4 + w) * 2 + 1]);
       }
+      if (sneg) {
+        const float t_lo = lo;
+        lo = -hi;
+        hi = -t_lo;
+      }
       if (kQuant) {
         const TokenGrid g = token_grid(lo, hi, rs, p.clip);
         if (quad == 0 && lane == 0) {
@@ -679,10 +706,10 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
           p.zero[t] = g.zero;
         }
         if (active)
-          quant_store<kPairs>(v, make_float2(g.c, odd_neg ? -g.c : g.c), g.zm, g.clamp,
+          quant_store<kPairs>(v, make_float2(sneg ? -g.c : g.c, (sneg != odd_neg) ? -g.c : g.c), g.zm, g.clamp,
                               p.q + static_cast<int64_t>(t) * (p.n >> 1) + (j0 >> 1));
       } else if (active) {
-        store_y<kPairs>(v, rs, p.y + static_cast<int64_t>(t) * p.ldy + j0, odd_neg ? -rs : rs);
+        store_y<kPairs>(v, sneg ? -rs : rs, p.y + static_cast<int64_t>(t) * p.ldy + j0, (sneg != odd_neg) ? -rs : rs);
       }
     }
   }
@@ -784,7 +811,8 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
   float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [token parity][half][quadrant][lo, hi]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const SignPlan sp = make_plan<kF28, kNcol>(p);
+  const OutlierRef orf = load_outlier(p);
+  const SignPlan sp = make_plan<kF28, kNcol>(p, orf);
   const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
   const uint32_t seg_xor = (col_xor >> 3) & 7u;
   const int box_xor = static_cast<int>(col_xor >> 6);
@@ -925,6 +953,7 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
       }
     }
     const float rs = p.inv_sqrt_n;
+    const bool sneg = outlier_sigma_neg(p, sp, orf);  // every output negated
     const bool odd_neg = (col_xor & 1u) != 0;  // see rotq_stream_kernel
     bool live = true;
     int i = 0;
@@ -981,6 +1010,11 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
         lo = fminf(lo, rslot[w * 2]);
         hi = fmaxf(hi, rslot[w * 2 + 1]);
       }
+      if (sneg) {
+        const float t_lo = lo;
+        lo = -hi;
+        hi = -t_lo;
+      }
       if (kQuant) {
         const TokenGrid g = token_grid(lo, hi, rs, p.clip);
         if (warp == 0 && lane == 0) {
@@ -988,10 +1022,10 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
           p.zero[t] = g.zero;
         }
         if (active)
-          quant_store<kPairs>(v, make_float2(g.c, odd_neg ? -g.c : g.c), g.zm, g.clamp,
+          quant_store<kPairs>(v, make_float2(sneg ? -g.c : g.c, (sneg != odd_neg) ? -g.c : g.c), g.zm, g.clamp,
                               p.q + static_cast<int64_t>(t) * (p.n >> 1) + (j0 >> 1));
       } else if (active) {
-        store_y<kPairs>(v, rs, p.y + static_cast<int64_t>(t) * p.ldy + j0, odd_neg ? -rs : rs);
+        store_y<kPairs>(v, sneg ? -rs : rs, p.y + static_cast<int64_t>(t) * p.ldy + j0, (sneg != odd_neg) ? -rs : rs);
       }
     }
   }
