@@ -394,8 +394,8 @@ struct TokenGrid {
 };
 
 __device__ __forceinline__ TokenGrid token_grid(float lo_w, float hi_w, float rs, float clip) {
-  // The grid sits on every token's critical path, so it avoids the second IEEE division: scale is
-  // the exact fp32 quotient (u - l) / 15; zero = rne(-l / scale) comes from -l * (1 / scale),
+  // The grid sits on every token's critical path, so it avoids IEEE divisions: scale is the exact
+  // fp32 quotient (u - l) / 15; zero = rne(-l / scale) comes from -l * (1 / scale),
   // which lies within a few ulps of the exact fp32 quotient -- only when that puts it within a
   // guard band of a half-integer could the two round differently, and only then is the exact
   // division taken. 1 / scale itself (for the codes) is the hardware approximation.
@@ -408,12 +408,17 @@ __device__ __forceinline__ TokenGrid token_grid(float lo_w, float hi_w, float rs
     tg.zero = rintf(-l);
     inv = 1.f;
   } else {
-    tg.scale = __fdiv_rn(__fsub_rn(u, l), 15.f);
+    // (u - l) / 15 rounded to nearest: x * fp32(1/15) with one FMA correction step, which equals
+    // the IEEE quotient for every finite fp32 x except -0 (checked on the GPU over all 2^32
+    // patterns; here x = u - l > 0, and an infinite range keeps its quotient, infinity)
+    const float d = __fsub_rn(u, l);
+    const float q0 = __fmul_rn(d, 1.0f / 15.0f);
+    tg.scale = isinf(d) ? d : __fmaf_rn(__fmaf_rn(-q0, 15.0f, d), 1.0f / 15.0f, q0);
     asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(tg.scale));
-    const float q0 = __fmul_rn(-l, inv);
-    tg.zero = rintf(q0);
-    const float off = fabsf(__fsub_rn(q0, tg.zero));      // distance to the nearest integer
-    const float guard = fmaf(fabsf(q0), 0x1p-19f, 0x1p-40f);  // ~16 ulps of q0
+    const float z0 = __fmul_rn(-l, inv);
+    tg.zero = rintf(z0);
+    const float off = fabsf(__fsub_rn(z0, tg.zero));      // distance to the nearest integer
+    const float guard = fmaf(fabsf(z0), 0x1p-19f, 0x1p-40f);  // ~16 ulps of z0
     if (!(0.5f - off > guard)) tg.zero = rintf(__fdiv_rn(-l, tg.scale));
   }
   tg.c = __fmul_rn(rs, inv);
