@@ -39,6 +39,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "signrot_device.cuh"
 #include "signrot_internal.h"
@@ -499,7 +500,6 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
   float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [buffer][4 quadrants][lo, hi]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const OutlierRef orf = load_outlier(p);  // issued ahead of the bulk copies
   if (threadIdx.x == 0) {
     for (int i = 0; i < S * kDW; ++i) mbar_init(smem_u32(&lfull[i]), 1);
     for (int i = 0; i < kTiles; ++i) {
@@ -513,6 +513,10 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
     fence_mbar_init();
   }
   __syncthreads();
+  // everything above touched only this CTA's shared memory; inputs may come from the grid before
+  griddep_wait();
+  griddep_launch_dependents();
+  const OutlierRef orf = load_outlier(p);  // issued ahead of the bulk copies
 
   // D warp w's share of the row: lane chunks [c0, c0 + 32 * per) of the kRowChunks
   const bool dwarp = warp >= kDWarp0 && warp < kMmaWarp;
@@ -816,6 +820,8 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
   float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [token parity][half][quadrant][lo, hi]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_wait();  // inputs may come from the grid before
+  griddep_launch_dependents();
   const OutlierRef orf = load_outlier(p);
   const SignPlan sp = make_plan<kF28, kNcol>(p, orf);
   const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
@@ -1045,6 +1051,23 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
 
 // ------------------------------------------------------------------------------------- host
 
+// Launch with programmatic stream serialization: the kernel may be scheduled while the previous
+// kernel in the stream is finishing; it waits (griddepcontrol.wait) before reading any input.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int threads, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -1076,9 +1099,9 @@ cudaError_t launch_wide(const CUtensorMap& tmap, const TcParams& p0, cudaStream_
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int grid = p.T < sms ? p.T : sms;
-  kern<<<grid, kWideThreads, smem, st>>>(tmap, p);
+  e = launch_pdl(kern, grid, kWideThreads, smem, st, tmap, p);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 template <bool kF28>
@@ -1105,9 +1128,9 @@ cudaError_t launch_stream(const TcParams& p0, cudaStream_t st) {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int grid = p.T < sms ? p.T : sms;
-  kern<<<grid, stream_threads(kNcol), smem, st>>>(p);
+  e = launch_pdl(kern, grid, stream_threads(kNcol), smem, st, p);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 template <int kNcol, bool kF28>

@@ -25,6 +25,10 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+// Programmatic dependent launch: block until the grids this one depends on have completed and
+// their writes are visible; let the next grid in the stream start launching its CTAs.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 // Shared-memory counter with acquire-release ordering: the writes a warp made (and fenced for the
 // async proxy) before its increment are visible to the warp that reads the final count.
 __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* ctr, uint32_t v) {
