@@ -227,6 +227,15 @@ __device__ __forceinline__ void fwht_local(float2 (&p)[kPairs]) {
 
 // D's signs of one 16-byte chunk (8 bf16 columns, D at d8[0..8)) as XOR masks on its four
 // 32-bit words.
+__device__ __forceinline__ uint4 chunk_sign_masks(uint2 d8) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t pair = ((i < 2 ? d8.x : d8.y) >> (16 * (i & 1))) & 0xffffu;  // d[2i], d[2i+1]
+    w[i] = ((pair & 0x80u) << 8) | ((pair & 0x8000u) << 16);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
 __device__ __forceinline__ uint4 chunk_sign_masks(const int8_t* d8) {
   uint32_t w[4];
 #pragma unroll
@@ -531,9 +540,24 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
     mbar_arrive_expect_tx(fb, part_bytes);
     bulk_load(smem_u32(lin + st * kRowBytes + c0 * 16), xpart + static_cast<int64_t>(t) * p.ldx * 2, part_bytes, fb);
   };
+  // The D warps' sign words are loaded (8 bytes per chunk when D is 8-byte aligned) before the
+  // bulk copies are issued, so that they do not queue behind every CTA's first copies; the mask
+  // arithmetic on them comes after the copies are on their way.
+  const int M = kF28 ? (1 << p.logM) : 0;
+  const bool last = per == kPerD;  // this warp also takes its lanes' kPerD-th chunk
+  const bool d_aligned = (reinterpret_cast<uintptr_t>(p.d) & 7u) == 0;
+  uint2 draw[kPerD];
+  if (dwarp && d_aligned) {
+#pragma unroll
+    for (int u = 0; u < kPerD; ++u) {
+      const int L = (u < per ? c0 + 32 * u : c0) + lane;
+      const int k = L / (kNcol / 8), b0 = (L % (kNcol / 8)) * 8;
+      const int j0 = kF28 ? (k >> 2) * M + (k & 3) * kNcol + b0 : k * kNcol + b0;
+      draw[u] = *reinterpret_cast<const uint2*>(p.d + j0);
+    }
+  }
   int issued = 0;  // bulk copies this D warp has started (lane 0)
   if (dwarp && lane == 0) {
-    // start streaming before the A matrix and the masks are built
     for (int st = 0; st < S; ++st) {
       const int t = blockIdx.x + st * gridDim.x;
       if (t >= p.T) break;
@@ -544,9 +568,6 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
 
   const SignPlan sp = make_plan<kF28, kNcol>(p, orf);
   const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
-  const int M = kF28 ? (1 << p.logM) : 0;
-  // D warps: their sign masks and tile destinations (global loads of D) ...
-  const bool last = per == kPerD;  // this warp also takes its lanes' kPerD-th chunk
   uint4 mask[kPerD];
   uint32_t dst[kPerD];
   if (dwarp) {
@@ -555,7 +576,12 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
       const int L = (u < per ? c0 + 32 * u : c0) + lane;
       const int k = L / (kNcol / 8), b0 = (L % (kNcol / 8)) * 8;
       const int j0 = kF28 ? (k >> 2) * M + (k & 3) * kNcol + b0 : k * kNcol + b0;
-      mask[u] = chunk_sign_masks(p.d + j0);
+      if (d_aligned) {
+        asm volatile("" : "+r"(draw[u].x), "+r"(draw[u].y));  // keeps the use after the copies
+        mask[u] = chunk_sign_masks(draw[u]);
+      } else {
+        mask[u] = chunk_sign_masks(p.d + j0);
+      }
       const int bp = b0 ^ static_cast<int>(col_xor & ~7u);  // where this chunk's columns go
       const int nbp = bp >> 6, segp = (bp >> 3) & 7;
       dst[u] = static_cast<uint32_t>(nbp) * kChunkBytes + k * 128 + ((segp ^ (k & 7)) << 4);
