@@ -870,6 +870,7 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
   const bool dwarp = warp >= kDWarp0 && warp < kTmaWarp;
   const int td = threadIdx.x - kDWarp0 * 32;
   uint32_t bits[kPerD];
+  const bool d_aligned = (reinterpret_cast<uintptr_t>(p.d) & 7u) == 0;
   if (dwarp) {
     // D signs of this lane's chunks, in the staged tile's order: chunk ch holds row (K index)
     // ch % (kKRows * 8) / 8, input columns of box (nb ^ box_xor), segment (slot ^ row) & 7
@@ -881,8 +882,14 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
       const int b0 = (nb ^ box_xor) * 64 + ((slot ^ (row & 7)) << 3);
       const int j0 = kF28 ? (row >> 2) * M + (row & 3) * kNcol + b0 : row * kNcol + b0;
       uint32_t b = 0;
+      if (d_aligned) {
+        const uint2 w = *reinterpret_cast<const uint2*>(p.d + j0);  // 8 signs in one load
 #pragma unroll
-      for (int e = 0; e < 8; ++e) b |= (p.d[j0 + e] < 0 ? 1u : 0u) << (15 + 16 * (e & 1) - (e >> 1));
+        for (int e = 0; e < 8; ++e) b |= (((e < 4 ? w.x : w.y) >> (8 * (e & 3) + 7)) & 1u) << (15 + 16 * (e & 1) - (e >> 1));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) b |= (p.d[j0 + e] < 0 ? 1u : 0u) << (15 + 16 * (e & 1) - (e >> 1));
+      }
       bits[u] = b;
     }
   } else {
