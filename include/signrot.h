@@ -133,8 +133,10 @@ signrot_status signrot_rotate(const void* x, int32_t dtype, int64_t T, int32_t n
  *   code_j = clamp(rne(y_j / scale[t]) + zero[t], 0, 15)       (rne: nearest, ties to even)
  *   a row with hi == lo gets scale = 1, zero = rne(-lo).
  * q[t * (n / 2) + i] = code_{2i} | code_{2i+1} << 4 (uint8, device, [T, n/2] row-major; n even).
- * Dequantize with (code - zero) * scale. bits must be 4; clip in (0, 1] (1 = no clipping, as in
- * the worked example). s may be NULL (plain rotation, no sign adjustment).
+ * Dequantize with (code - zero) * scale. clip in (0, 1] (1 = no clipping, as in the worked
+ * example). s may be NULL (plain rotation, no sign adjustment).
+ * bits = 8 gives the same grid with 255 levels (/ 255 and clamp(., 0, 255) above) and one code per
+ * byte: q[t * n + j] = code_j ([T, n]). Any other bits -> SIGNROT_ERR_UNSUPPORTED.
  * The codes are decided in fp32 with the reciprocal of the scale, so a code may differ by one
  * from the formula above where y / scale lies within an ulp of a half-integer.
  */
@@ -159,6 +161,26 @@ signrot_status signrot_rotate_quant_outlier(const void* x, int32_t dtype, int64_
                                             int64_t ld, const int8_t* d, const int32_t* k,
                                             const float* xk, int32_t bits, float clip, uint8_t* q,
                                             float* scale, float* zero, void* stream);
+
+/*
+ * signrot_rotate_quant_sym / signrot_rotate_quant_sym_outlier -- the same path with the
+ * symmetric per-token grid instead (the explainer's comparison grid, "Worked example": levels
+ * spaced evenly on both sides of zero): L = 2^(bits-1) - 1 (7 for bits = 4, 127 for bits = 8),
+ *   scale[t] = max_j |y_j| / L  (1 for an all-zero row),  code_j = clamp(rne(y_j / scale[t]), -L, L).
+ * bits = 4: q [T, n/2], q[t * (n/2) + i] = (code_{2i} & 15) | (code_{2i+1} & 15) << 4 (two's
+ * complement nibbles); bits = 8: q [T, n] as int8. No zero-point and no clip. The sign
+ * adjustment is s (or NULL) or, in the _outlier form, k and xk as for
+ * signrot_rotate_quant_outlier. Codes are decided as in signrot_rotate_quant (reciprocal of the
+ * scale on the fused kernel: a code may differ by one where y / scale is within an ulp of a
+ * half-integer).
+ */
+signrot_status signrot_rotate_quant_sym(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                        const int8_t* d, const int8_t* s, int32_t bits, uint8_t* q,
+                                        float* scale, void* stream);
+signrot_status signrot_rotate_quant_sym_outlier(const void* x, int32_t dtype, int64_t T, int32_t n,
+                                                int64_t ld, const int8_t* d, const int32_t* k,
+                                                const float* xk, int32_t bits, uint8_t* q, float* scale,
+                                                void* stream);
 
 /*
  * signrot_rotate_quant_host -- the fused path between HOST buffers: x_host [T, ld] (pinned for

@@ -8,7 +8,8 @@
 //   2. H_28 across the stride-M axis (dense 28 x 28 block, F = 28 only)
 //   3. FWHT of length M along the contiguous axis, radix-2 stages
 //   4. y = s (.) w / sqrt(n), rounded once to fp32
-//   5. check path: store y; quantized path: row min/max, scale, zero, codes, nibble pack.
+//   5. check path: store y; quantized path: row min/max, the asymmetric (scale, zero) or symmetric
+//      (scale) grid, codes packed two per byte (4 bits) or one per byte (8 bits).
 // The rotation accumulates in fp64 (fp32 only for n = 32768, whose fp64 row would not fit in
 // shared memory), so y is the correctly rounded fp32 of the exact rotation up to a rare double
 // rounding, and the quantizer then takes the same fp32 steps as the formula in the header
@@ -127,16 +128,39 @@ __global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, 
     }
     if (kQuant) {
       block_minmax(lo, hi, red);
-      const QuantGrid g = make_grid(lo, hi, a.clip);
-      if (threadIdx.x == 0) {
-        a.scale[t] = g.scale;
-        a.zero[t] = g.zero;
-      }
-      uint8_t* qr = a.q + t * (n >> 1);
-      for (int i = threadIdx.x; i < (n >> 1); i += blockDim.x) {
-        const uint32_t c0 = quant_code_div(ybuf[2 * i], g);
-        const uint32_t c1 = quant_code_div(ybuf[2 * i + 1], g);
-        qr[i] = static_cast<uint8_t>(c0 | (c1 << 4));
+      if (a.sym) {
+        const float L = a.bits == 8 ? 127.f : 7.f;
+        const float scale = sym_scale(lo, hi, L);
+        if (threadIdx.x == 0) a.scale[t] = scale;
+        if (a.bits == 8) {
+          int8_t* qr = reinterpret_cast<int8_t*>(a.q) + t * n;
+          for (int j = threadIdx.x; j < n; j += blockDim.x) qr[j] = static_cast<int8_t>(sym_code_div(ybuf[j], scale, L));
+        } else {
+          uint8_t* qr = a.q + t * (n >> 1);
+          for (int i = threadIdx.x; i < (n >> 1); i += blockDim.x) {
+            const uint32_t c0 = static_cast<uint32_t>(sym_code_div(ybuf[2 * i], scale, L)) & 15u;
+            const uint32_t c1 = static_cast<uint32_t>(sym_code_div(ybuf[2 * i + 1], scale, L)) & 15u;
+            qr[i] = static_cast<uint8_t>(c0 | (c1 << 4));
+          }
+        }
+      } else {
+        const float qmax = a.bits == 8 ? 255.f : 15.f;
+        const QuantGrid g = make_grid(lo, hi, a.clip, qmax);
+        if (threadIdx.x == 0) {
+          a.scale[t] = g.scale;
+          a.zero[t] = g.zero;
+        }
+        if (a.bits == 8) {
+          uint8_t* qr = a.q + t * n;
+          for (int j = threadIdx.x; j < n; j += blockDim.x) qr[j] = static_cast<uint8_t>(quant_code_div(ybuf[j], g, qmax));
+        } else {
+          uint8_t* qr = a.q + t * (n >> 1);
+          for (int i = threadIdx.x; i < (n >> 1); i += blockDim.x) {
+            const uint32_t c0 = quant_code_div(ybuf[2 * i], g);
+            const uint32_t c1 = quant_code_div(ybuf[2 * i + 1], g);
+            qr[i] = static_cast<uint8_t>(c0 | (c1 << 4));
+          }
+        }
       }
     }
     __syncthreads();

@@ -336,19 +336,30 @@ __device__ __forceinline__ void local_minmax_xy(const float2 (&p)[kPairs], float
 
 
 // Eight consecutive codes -> one u32 of nibbles (element 2i low nibble). u holds the bit
-// patterns of fma(w, c, zero + 1.5*2^23), whose low byte is the code (0..15).
+// patterns of fma(w, c, zero + 1.5*2^23), whose low byte is the code: 0..15 on the asymmetric grid,
+// where one multiply-add per pair combines them; -7..7 (two's complement) on the symmetric grid,
+// whose negative codes carry set high bits into the byte and are masked to their nibble first.
+template <bool kSigned = false>
 __device__ __forceinline__ uint32_t pack8(const uint32_t (&u)[8]) {
-  const uint32_t b01 = u[1] * 16u + u[0], b23 = u[3] * 16u + u[2];
-  const uint32_t b45 = u[5] * 16u + u[4], b67 = u[7] * 16u + u[6];
-  const uint32_t w0 = b23 * 256u + b01, w1 = b67 * 256u + b45;
-  return __byte_perm(w0, w1, 0x5410);
+  if constexpr (kSigned) {
+    uint32_t b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) b[i] = ((u[2 * i + 1] & 15u) << 4) | (u[2 * i] & 15u);
+    return __byte_perm(b[0] | (b[1] << 8), b[2] | (b[3] << 8), 0x5410);
+  } else {
+    const uint32_t b01 = u[1] * 16u + u[0], b23 = u[3] * 16u + u[2];
+    const uint32_t b45 = u[5] * 16u + u[4], b67 = u[7] * 16u + u[6];
+    const uint32_t w0 = b23 * 256u + b01, w1 = b67 * 256u + b45;
+    return __byte_perm(w0, w1, 0x5410);
+  }
 }
 
-// Quantize 16 pairs (32 consecutive columns) into one 16-byte store of packed nibbles.
-template <bool kClamp>
-__device__ __forceinline__ uint4 quant16(const float2* p, float2 c2, float zm) {
+// Quantize 16 pairs (32 consecutive columns) into one 16-byte store of packed nibbles. Each
+// fma(w, c, zm) lands in [lo_m, hi_m] around 1.5 * 2^23 after clamping, where the fp32 ulp is 1,
+// so its low bits are the code (two's complement for the symmetric grid's negative codes).
+template <bool kClamp, bool kSigned>
+__device__ __forceinline__ uint4 quant16(const float2* p, float2 c2, float zm, float lo_m, float hi_m) {
   const float2 z2 = make_float2(zm, zm);
-  const float lo_m = kMagic, hi_m = kMagic + 15.f;
   uint32_t words[4];
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
@@ -363,23 +374,55 @@ __device__ __forceinline__ uint4 quant16(const float2* p, float2 c2, float zm) {
       u[2 * k] = __float_as_uint(t.x);
       u[2 * k + 1] = __float_as_uint(t.y);
     }
-    words[g] = pack8(u);
+    words[g] = pack8<kSigned>(u);
   }
   return make_uint4(words[0], words[1], words[2], words[3]);
 }
 
-// Quantize + store one run of 2*kPairs consecutive channels at q_out (16 B aligned); c2 holds the
-// multipliers of the even and the odd channels.
-template <int kPairs>
-__device__ __forceinline__ void quant_store(const float2 (&p)[kPairs], float2 c2, float zm, bool clamp,
-                                            uint8_t* q_out) {
+// The 8-bit form: 8 pairs (16 consecutive columns) into one 16-byte store, one code per byte.
+template <bool kClamp>
+__device__ __forceinline__ uint4 quant16_bytes(const float2* p, float2 c2, float zm, float lo_m, float hi_m) {
+  const float2 z2 = make_float2(zm, zm);
+  uint32_t words[4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float2 t0 = __ffma2_rn(p[2 * g], c2, z2), t1 = __ffma2_rn(p[2 * g + 1], c2, z2);
+    if (kClamp) {
+      t0.x = fminf(fmaxf(t0.x, lo_m), hi_m);
+      t0.y = fminf(fmaxf(t0.y, lo_m), hi_m);
+      t1.x = fminf(fmaxf(t1.x, lo_m), hi_m);
+      t1.y = fminf(fmaxf(t1.y, lo_m), hi_m);
+    }
+    const uint32_t w01 = __byte_perm(__float_as_uint(t0.x), __float_as_uint(t0.y), 0x0040);
+    const uint32_t w23 = __byte_perm(__float_as_uint(t1.x), __float_as_uint(t1.y), 0x0040);
+    words[g] = __byte_perm(w01, w23, 0x5410);
+  }
+  return make_uint4(words[0], words[1], words[2], words[3]);
+}
+
+// Quantize + store one run of 2*kPairs consecutive channels at q_out (16 B aligned): kBits = 4,
+// two codes per byte (element 2i low nibble); kBits = 8, one per byte. c2 holds the multipliers of
+// the even and the odd channels.
+template <int kPairs, int kBits, bool kSigned>
+__device__ __forceinline__ void quant_store(const float2 (&p)[kPairs], float2 c2, float zm, bool clamp, float lo_m,
+                                            float hi_m, uint8_t* q_out) {
   uint4* dst = reinterpret_cast<uint4*>(q_out);
-  if (clamp) {
+  if constexpr (kBits == 4) {
+    if (clamp) {
 #pragma unroll
-    for (int i = 0; i < kPairs / 16; ++i) dst[i] = quant16<true>(p + 16 * i, c2, zm);
+      for (int i = 0; i < kPairs / 16; ++i) dst[i] = quant16<true, kSigned>(p + 16 * i, c2, zm, lo_m, hi_m);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kPairs / 16; ++i) dst[i] = quant16<false, kSigned>(p + 16 * i, c2, zm, lo_m, hi_m);
+    }
   } else {
+    if (clamp) {
 #pragma unroll
-    for (int i = 0; i < kPairs / 16; ++i) dst[i] = quant16<false>(p + 16 * i, c2, zm);
+      for (int i = 0; i < kPairs / 8; ++i) dst[i] = quant16_bytes<true>(p + 8 * i, c2, zm, lo_m, hi_m);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kPairs / 8; ++i) dst[i] = quant16_bytes<false>(p + 8 * i, c2, zm, lo_m, hi_m);
+    }
   }
 }
 
@@ -398,14 +441,16 @@ __device__ __forceinline__ void store_y(const float2 (&p)[kPairs], float rs, flo
 struct TokenGrid {
   float c;      // w -> y / scale
   float zm;     // zero + 1.5 * 2^23
-  bool clamp;   // some code of this token falls outside [0, 15] before clamping
+  bool clamp;   // some code of this token falls outside [code_min, code_max] before clamping
   float scale;
   float zero;
+  float lo_m, hi_m;  // 1.5 * 2^23 + code_min, 1.5 * 2^23 + code_max: the clamp bounds of fma(w, c, zm)
 };
 
-__device__ __forceinline__ TokenGrid token_grid(float lo_w, float hi_w, float rs, float clip) {
+// Asymmetric grid with codes 0 .. qmax (15 or 255) over [clip * min y, clip * max y].
+__device__ __forceinline__ TokenGrid token_grid(float lo_w, float hi_w, float rs, float clip, float qmax) {
   // The grid sits on every token's critical path, so it avoids IEEE divisions: scale is the exact
-  // fp32 quotient (u - l) / 15; zero = rne(-l / scale) comes from -l * (1 / scale),
+  // fp32 quotient (u - l) / qmax; zero = rne(-l / scale) comes from -l * (1 / scale),
   // which lies within a few ulps of the exact fp32 quotient -- only when that puts it within a
   // guard band of a half-integer could the two round differently, and only then is the exact
   // division taken. 1 / scale itself (for the codes) is the hardware approximation.
@@ -418,12 +463,16 @@ __device__ __forceinline__ TokenGrid token_grid(float lo_w, float hi_w, float rs
     tg.zero = rintf(-l);
     inv = 1.f;
   } else {
-    // (u - l) / 15 rounded to nearest: x * fp32(1/15) with one FMA correction step, which equals
-    // the IEEE quotient for every finite fp32 x except -0 (checked on the GPU over all 2^32
-    // patterns; here x = u - l > 0, and an infinite range keeps its quotient, infinity)
     const float d = __fsub_rn(u, l);
-    const float q0 = __fmul_rn(d, 1.0f / 15.0f);
-    tg.scale = isinf(d) ? d : __fmaf_rn(__fmaf_rn(-q0, 15.0f, d), 1.0f / 15.0f, q0);
+    if (qmax == 15.f) {
+      // (u - l) / 15 rounded to nearest: x * fp32(1/15) with one FMA correction step, which
+      // equals the IEEE quotient for every finite fp32 x except -0 (checked on the GPU over all
+      // 2^32 patterns; here x = u - l > 0, and an infinite range keeps its quotient, infinity)
+      const float q0 = __fmul_rn(d, 1.0f / 15.0f);
+      tg.scale = isinf(d) ? d : __fmaf_rn(__fmaf_rn(-q0, 15.0f, d), 1.0f / 15.0f, q0);
+    } else {
+      tg.scale = __fdiv_rn(d, qmax);
+    }
     asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(tg.scale));
     const float z0 = __fmul_rn(-l, inv);
     tg.zero = rintf(z0);
@@ -433,12 +482,64 @@ __device__ __forceinline__ TokenGrid token_grid(float lo_w, float hi_w, float rs
   }
   tg.c = __fmul_rn(rs, inv);
   tg.zm = __fadd_rn(tg.zero, kMagic);
+  tg.lo_m = kMagic;
+  tg.hi_m = kMagic + qmax;
   // codes are monotone in w, so the row's extremes decide whether any code needs clamping;
   // a zero-point too large for the 1.5 * 2^23 trick also takes the clamped path
   const int c_lo = static_cast<int>(__float_as_uint(fmaf(lo_w, tg.c, tg.zm)) - __float_as_uint(kMagic));
   const int c_hi = static_cast<int>(__float_as_uint(fmaf(hi_w, tg.c, tg.zm)) - __float_as_uint(kMagic));
-  tg.clamp = !(c_lo >= 0 && c_hi <= 15) || fabsf(tg.zero) > 4194304.f;
+  tg.clamp = !(c_lo >= 0 && c_hi <= static_cast<int>(qmax)) || fabsf(tg.zero) > 4194304.f;
   return tg;
+}
+
+// Symmetric grid: codes -L .. L (L = 7 or 127), scale = max |y| / L (1 for an all-zero row),
+// code = clamp(rne(y / scale), -L, L); no zero-point.
+__device__ __forceinline__ TokenGrid token_grid_sym(float lo_w, float hi_w, float rs, float L) {
+  const float lo_y = __fmul_rn(lo_w, rs), hi_y = __fmul_rn(hi_w, rs);
+  const float amax = fmaxf(fabsf(lo_y), fabsf(hi_y));
+  TokenGrid tg;
+  tg.scale = amax == 0.f ? 1.f : __fdiv_rn(amax, L);
+  float inv;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(tg.scale));
+  tg.c = __fmul_rn(rs, inv);
+  tg.zero = 0.f;
+  tg.zm = kMagic;
+  tg.lo_m = kMagic - L;
+  tg.hi_m = kMagic + L;
+  const int c_lo = static_cast<int>(__float_as_uint(fmaf(lo_w, tg.c, kMagic)) - __float_as_uint(kMagic));
+  const int c_hi = static_cast<int>(__float_as_uint(fmaf(hi_w, tg.c, kMagic)) - __float_as_uint(kMagic));
+  tg.clamp = !(c_lo >= -static_cast<int>(L) && c_hi <= static_cast<int>(L));
+  return tg;
+}
+
+// What a fused kernel writes per token: the check path's fp32 y, or codes of one grid.
+enum : int { kModeY = 0, kModeA4 = 1, kModeA8 = 2, kModeS4 = 3, kModeS8 = 4 };
+__host__ __device__ constexpr int mode_bits(int m) { return (m == kModeA8 || m == kModeS8) ? 8 : 4; }
+__host__ __device__ constexpr bool mode_sym(int m) { return m == kModeS4 || m == kModeS8; }
+
+// The end of one token for one thread's run of 2 * kPairs output channels starting at channel j0:
+// grid from the token's extremes, codes (or y) stored. sneg / odd_neg: every output / every odd
+// column comes out of the transform negated (see rotq_stream_kernel). writer: this thread also
+// stores the token's scale and zero-point.
+template <int kPairs, int kMode>
+__device__ __forceinline__ void finish_token(const float2 (&v)[kPairs], float lo, float hi, bool sneg, bool odd_neg,
+                                             bool active, bool writer, const TcParams& p, int t, int64_t j0) {
+  const float rs = p.inv_sqrt_n;
+  if constexpr (kMode == kModeY) {
+    if (active) store_y<kPairs>(v, sneg ? -rs : rs, p.y + static_cast<int64_t>(t) * p.ldy + j0, (sneg != odd_neg) ? -rs : rs);
+  } else {
+    constexpr int kBits = mode_bits(kMode);
+    const TokenGrid g = mode_sym(kMode) ? token_grid_sym(lo, hi, rs, kBits == 4 ? 7.f : 127.f)
+                                        : token_grid(lo, hi, rs, p.clip, kBits == 4 ? 15.f : 255.f);
+    if (writer) {
+      p.scale[t] = g.scale;
+      if (!mode_sym(kMode)) p.zero[t] = g.zero;
+    }
+    if (active)
+      quant_store<kPairs, kBits, mode_sym(kMode)>(
+          v, make_float2(sneg ? -g.c : g.c, (sneg != odd_neg) ? -g.c : g.c), g.zm, g.clamp, g.lo_m, g.hi_m,
+          p.q + static_cast<int64_t>(t) * (p.n * kBits / 8) + j0 * kBits / 8);
+  }
 }
 
 // ------------------------------------------------------------------------------------- kernel
@@ -464,7 +565,7 @@ constexpr int kStreamDWarps = 3;
 constexpr int kStreamTiles = 3;
 __host__ __device__ constexpr int stream_threads(int ncol) { return 32 * (4 * epi_groups(ncol) + kStreamDWarps + 1); }
 
-template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
+template <int kNcol, bool kF28, bool kVecSign, int kMode>
 __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(TcParams p) {
   static_assert(kNcol <= 128, "the streamed variant keeps a token's lane line in registers");
   constexpr int kKRows = kF28 ? 112 : 128;
@@ -682,7 +783,6 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
         sbits[w] = b;
       }
     }
-    const float rs = p.inv_sqrt_n;
     // the outlier permutation's bit 0 is not applied to the input: every odd column of the
     // transform comes out negated (H P_1 = diag((-1)^j) H), which min/max and quantization undo
     const bool sneg = outlier_sigma_neg(p, sp, orf);  // every output negated
@@ -734,18 +834,7 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
         lo = -hi;
         hi = -t_lo;
       }
-      if (kQuant) {
-        const TokenGrid g = token_grid(lo, hi, rs, p.clip);
-        if (quad == 0 && lane == 0) {
-          p.scale[t] = g.scale;
-          p.zero[t] = g.zero;
-        }
-        if (active)
-          quant_store<kPairs>(v, make_float2(sneg ? -g.c : g.c, (sneg != odd_neg) ? -g.c : g.c), g.zm, g.clamp,
-                              p.q + static_cast<int64_t>(t) * (p.n >> 1) + (j0 >> 1));
-      } else if (active) {
-        store_y<kPairs>(v, sneg ? -rs : rs, p.y + static_cast<int64_t>(t) * p.ldy + j0, (sneg != odd_neg) ? -rs : rs);
-      }
+      finish_token<kPairs, kMode>(v, lo, hi, sneg, odd_neg, active, quad == 0 && lane == 0, p, t, j0);
     }
   }
 
@@ -806,7 +895,7 @@ __device__ __forceinline__ void inplace_d_pass_bits(uint4* base, const uint32_t 
   }
 }
 
-template <bool kF28, bool kVecSign, bool kQuant>
+template <bool kF28, bool kVecSign, int kMode>
 __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                     TcParams p) {
   constexpr int kNcol = 256, kHalf = 128, kPairs = 64;
@@ -996,7 +1085,6 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
         sbits[w] = b;
       }
     }
-    const float rs = p.inv_sqrt_n;
     const bool sneg = outlier_sigma_neg(p, sp, orf);  // every output negated
     const bool odd_neg = (col_xor & 1u) != 0;  // see rotq_stream_kernel
     bool live = true;
@@ -1059,18 +1147,7 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
         lo = -hi;
         hi = -t_lo;
       }
-      if (kQuant) {
-        const TokenGrid g = token_grid(lo, hi, rs, p.clip);
-        if (warp == 0 && lane == 0) {
-          p.scale[t] = g.scale;
-          p.zero[t] = g.zero;
-        }
-        if (active)
-          quant_store<kPairs>(v, make_float2(sneg ? -g.c : g.c, (sneg != odd_neg) ? -g.c : g.c), g.zm, g.clamp,
-                              p.q + static_cast<int64_t>(t) * (p.n >> 1) + (j0 >> 1));
-      } else if (active) {
-        store_y<kPairs>(v, sneg ? -rs : rs, p.y + static_cast<int64_t>(t) * p.ldy + j0, (sneg != odd_neg) ? -rs : rs);
-      }
+      finish_token<kPairs, kMode>(v, lo, hi, sneg, odd_neg, active, warp == 0 && lane == 0, p, t, j0);
     }
   }
 
@@ -1115,7 +1192,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <bool kF28, bool kVecSign, bool kQuant>
+template <bool kF28, bool kVecSign, int kMode>
 cudaError_t launch_wide(const CUtensorMap& tmap, const TcParams& p0, cudaStream_t st) {
   constexpr int kKRows = kF28 ? 112 : 128;
   constexpr uint32_t kStageBytes = 4 * kKRows * 128;
@@ -1125,7 +1202,7 @@ cudaError_t launch_wide(const CUtensorMap& tmap, const TcParams& p0, cudaStream_
   if (p.stages > 8) p.stages = 8;
   if (p.stages < 2) return cudaErrorNotSupported;
   const size_t smem = 1024 + kABytes + static_cast<size_t>(p.stages) * kStageBytes + 1024;
-  auto kern = rotq_wide_kernel<kF28, kVecSign, kQuant>;
+  auto kern = rotq_wide_kernel<kF28, kVecSign, kMode>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
@@ -1137,14 +1214,23 @@ cudaError_t launch_wide(const CUtensorMap& tmap, const TcParams& p0, cudaStream_
   return e;
 }
 
-template <bool kF28>
-cudaError_t dispatch_wide(const CUtensorMap& tmap, const TcParams& p, bool vec_sign, bool quant, cudaStream_t st) {
-  if (vec_sign)
-    return quant ? launch_wide<kF28, true, true>(tmap, p, st) : launch_wide<kF28, true, false>(tmap, p, st);
-  return quant ? launch_wide<kF28, false, true>(tmap, p, st) : launch_wide<kF28, false, false>(tmap, p, st);
+template <bool kF28, bool kVecSign>
+cudaError_t dispatch_wide_mode(const CUtensorMap& tmap, const TcParams& p, int mode, cudaStream_t st) {
+  switch (mode) {
+    case kModeY: return launch_wide<kF28, kVecSign, kModeY>(tmap, p, st);
+    case kModeA4: return launch_wide<kF28, kVecSign, kModeA4>(tmap, p, st);
+    case kModeA8: return launch_wide<kF28, kVecSign, kModeA8>(tmap, p, st);
+    case kModeS4: return launch_wide<kF28, kVecSign, kModeS4>(tmap, p, st);
+    default: return launch_wide<kF28, kVecSign, kModeS8>(tmap, p, st);
+  }
 }
 
-template <int kNcol, bool kF28, bool kVecSign, bool kQuant>
+template <bool kF28>
+cudaError_t dispatch_wide(const CUtensorMap& tmap, const TcParams& p, bool vec_sign, int mode, cudaStream_t st) {
+  return vec_sign ? dispatch_wide_mode<kF28, true>(tmap, p, mode, st) : dispatch_wide_mode<kF28, false>(tmap, p, mode, st);
+}
+
+template <int kNcol, bool kF28, bool kVecSign, int kMode>
 cudaError_t launch_stream(const TcParams& p0, cudaStream_t st) {
   constexpr int kKRows = kF28 ? 112 : 128;
   constexpr uint32_t kRowBytes = (kNcol / 64) * kKRows * 128;
@@ -1154,7 +1240,7 @@ cudaError_t launch_stream(const TcParams& p0, cudaStream_t st) {
   if (p.stages > 8) p.stages = 8;
   if (p.stages < 2) return cudaErrorNotSupported;
   const size_t smem = 1024 + kABytes + kStreamTiles * kRowBytes + static_cast<size_t>(p.stages) * kRowBytes + 1024;
-  auto kern = rotq_stream_kernel<kNcol, kF28, kVecSign, kQuant>;
+  auto kern = rotq_stream_kernel<kNcol, kF28, kVecSign, kMode>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
@@ -1166,11 +1252,20 @@ cudaError_t launch_stream(const TcParams& p0, cudaStream_t st) {
   return e;
 }
 
+template <int kNcol, bool kF28, bool kVecSign>
+cudaError_t dispatch_stream_mode(const TcParams& p, int mode, cudaStream_t st) {
+  switch (mode) {
+    case kModeY: return launch_stream<kNcol, kF28, kVecSign, kModeY>(p, st);
+    case kModeA4: return launch_stream<kNcol, kF28, kVecSign, kModeA4>(p, st);
+    case kModeA8: return launch_stream<kNcol, kF28, kVecSign, kModeA8>(p, st);
+    case kModeS4: return launch_stream<kNcol, kF28, kVecSign, kModeS4>(p, st);
+    default: return launch_stream<kNcol, kF28, kVecSign, kModeS8>(p, st);
+  }
+}
+
 template <int kNcol, bool kF28>
-cudaError_t dispatch_stream(const TcParams& p, bool vec_sign, bool quant, cudaStream_t st) {
-  if (vec_sign)
-    return quant ? launch_stream<kNcol, kF28, true, true>(p, st) : launch_stream<kNcol, kF28, true, false>(p, st);
-  return quant ? launch_stream<kNcol, kF28, false, true>(p, st) : launch_stream<kNcol, kF28, false, false>(p, st);
+cudaError_t dispatch_stream(const TcParams& p, bool vec_sign, int mode, cudaStream_t st) {
+  return vec_sign ? dispatch_stream_mode<kNcol, kF28, true>(p, mode, st) : dispatch_stream_mode<kNcol, kF28, false>(p, mode, st);
 }
 
 }  // namespace
@@ -1182,6 +1277,7 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
   if (ncol != 64 && ncol != 128 && ncol != 256) return cudaErrorNotSupported;
   if (reinterpret_cast<uintptr_t>(a.x) % 16 != 0 || a.ld % 8 != 0) return cudaErrorNotSupported;
   const bool quant = a.q != nullptr;
+  const int mode = !quant ? kModeY : (a.sym ? (a.bits == 8 ? kModeS8 : kModeS4) : (a.bits == 8 ? kModeA8 : kModeA4));
   if (quant && reinterpret_cast<uintptr_t>(a.q) % 16 != 0) return cudaErrorNotSupported;
   if (!quant && (reinterpret_cast<uintptr_t>(a.y) % 16 != 0 || a.ldy % 4 != 0)) return cudaErrorNotSupported;
   TcParams p{};
@@ -1204,8 +1300,8 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
   p.h = h;
   const bool vec = a.s != nullptr && a.kp == nullptr;
   // Up to 128 columns per token: the streamed kernel; 256 columns: the TMA-staged wide kernel.
-  if (ncol == 64) return f28 ? dispatch_stream<64, true>(p, vec, quant, st) : dispatch_stream<64, false>(p, vec, quant, st);
-  if (ncol == 128) return f28 ? dispatch_stream<128, true>(p, vec, quant, st) : dispatch_stream<128, false>(p, vec, quant, st);
+  if (ncol == 64) return f28 ? dispatch_stream<64, true>(p, vec, mode, st) : dispatch_stream<64, false>(p, vec, mode, st);
+  if (ncol == 128) return f28 ? dispatch_stream<128, true>(p, vec, mode, st) : dispatch_stream<128, false>(p, vec, mode, st);
 
   auto encode = encode_fn();
   if (encode == nullptr) return cudaErrorNotSupported;
@@ -1230,7 +1326,7 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   }
   if (r != CUDA_SUCCESS) return cudaErrorNotSupported;
-  return f28 ? dispatch_wide<true>(tmap, p, vec, quant, st) : dispatch_wide<false>(tmap, p, vec, quant, st);
+  return f28 ? dispatch_wide<true>(tmap, p, vec, mode, st) : dispatch_wide<false>(tmap, p, vec, mode, st);
 }
 
 cudaError_t read_device_error(uint32_t* out, bool clear) {

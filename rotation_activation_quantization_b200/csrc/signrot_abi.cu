@@ -164,16 +164,17 @@ signrot_status rotate_impl(const void* x, int32_t dtype, int64_t T, int32_t n, i
 signrot_status rotate_quant_impl(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
                                  const int8_t* d, const int8_t* s, const int32_t* kp, const float* xkp,
                                  int32_t bits, float clip, uint8_t* q, float* scale, float* zero,
-                                 void* stream) {
+                                 void* stream, bool sym = false) {
   g_last_error[0] = '\0';
   signrot::Shape sh;
   signrot_status st = check_rows(x, dtype, T, n, ld, &sh);
   if (st != SIGNROT_OK) return st;
-  if (bits != 4) return fail(SIGNROT_ERR_UNSUPPORTED, "bits = %d; only 4 is supported", bits);
+  if (bits != 4 && bits != 8) return fail(SIGNROT_ERR_UNSUPPORTED, "bits = %d; 4 and 8 are supported", bits);
   if (!(clip > 0.f && clip <= 1.f)) return fail(SIGNROT_ERR_UNSUPPORTED, "clip must lie in (0, 1]");
   if (d == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "d is NULL");
-  if (T > 0 && (q == nullptr || scale == nullptr || zero == nullptr))
-    return fail(SIGNROT_ERR_INVALID_ARG, "q, scale and zero must be device pointers");
+  if (T > 0 && (q == nullptr || scale == nullptr || (!sym && zero == nullptr)))
+    return fail(SIGNROT_ERR_INVALID_ARG, sym ? "q and scale must be device pointers"
+                                             : "q, scale and zero must be device pointers");
   if (!aligned(scale, 4) || !aligned(zero, 4))
     return fail(SIGNROT_ERR_ALIGNMENT, "scale / zero not 4-byte aligned");
   if (!aligned(kp, 4) || !aligned(xkp, 4)) return fail(SIGNROT_ERR_ALIGNMENT, "k or xk misaligned");
@@ -190,8 +191,10 @@ signrot_status rotate_quant_impl(const void* x, int32_t dtype, int64_t T, int32_
   a.xkp = xkp;
   a.q = q;
   a.scale = scale;
-  a.zero = zero;
+  a.zero = sym ? nullptr : zero;
   a.clip = clip;
+  a.bits = bits;
+  a.sym = sym;
   return run_rotate(a, static_cast<cudaStream_t>(stream));
 }
 
@@ -265,6 +268,19 @@ signrot_status signrot_rotate_quant_outlier(const void* x, int32_t dtype, int64_
                                             float* scale, float* zero, void* stream) {
   if (k == nullptr || xk == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "k and xk must be device pointers");
   return rotate_quant_impl(x, dtype, T, n, ld, d, nullptr, k, xk, bits, clip, q, scale, zero, stream);
+}
+
+signrot_status signrot_rotate_quant_sym(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                        const int8_t* d, const int8_t* s, int32_t bits, uint8_t* q, float* scale,
+                                        void* stream) {
+  return rotate_quant_impl(x, dtype, T, n, ld, d, s, nullptr, nullptr, bits, 1.f, q, scale, nullptr, stream, true);
+}
+
+signrot_status signrot_rotate_quant_sym_outlier(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                                const int8_t* d, const int32_t* k, const float* xk, int32_t bits,
+                                                uint8_t* q, float* scale, void* stream) {
+  if (k == nullptr || xk == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "k and xk must be device pointers");
+  return rotate_quant_impl(x, dtype, T, n, ld, d, nullptr, k, xk, bits, 1.f, q, scale, nullptr, stream, true);
 }
 
 size_t signrot_host_bytes_per_token(int32_t n, int32_t dtype) {

@@ -53,24 +53,34 @@ struct QuantGrid {
   float inv;    // fp32(1 / scale)
 };
 
-__device__ __forceinline__ QuantGrid make_grid(float lo, float hi, float clip) {
+__device__ __forceinline__ QuantGrid make_grid(float lo, float hi, float clip, float qmax = 15.f) {
   const float l = __fmul_rn(lo, clip), u = __fmul_rn(hi, clip);
   QuantGrid g;
   if (u == l) {
     g.scale = 1.f;
     g.zero = rintf(-l);
   } else {
-    g.scale = __fdiv_rn(__fsub_rn(u, l), 15.f);
+    g.scale = __fdiv_rn(__fsub_rn(u, l), qmax);
     g.zero = rintf(__fdiv_rn(-l, g.scale));
   }
   g.inv = __frcp_rn(g.scale);
   return g;
 }
 
-// code = clamp(rne(y / scale) + zero, 0, 15) with a true IEEE division (the formula as written).
-__device__ __forceinline__ uint32_t quant_code_div(float y, const QuantGrid& g) {
+// code = clamp(rne(y / scale) + zero, 0, qmax) with a true IEEE division (the formula as written).
+__device__ __forceinline__ uint32_t quant_code_div(float y, const QuantGrid& g, float qmax = 15.f) {
   const float v = __fadd_rn(rintf(__fdiv_rn(y, g.scale)), g.zero);
-  return static_cast<uint32_t>(fminf(fmaxf(v, 0.f), 15.f));
+  return static_cast<uint32_t>(fminf(fmaxf(v, 0.f), qmax));
+}
+
+// Symmetric grid, codes -L .. L: scale = max |y| / L (1 for an all-zero row) ...
+__device__ __forceinline__ float sym_scale(float lo, float hi, float L) {
+  const float amax = fmaxf(fabsf(lo), fabsf(hi));
+  return amax == 0.f ? 1.f : __fdiv_rn(amax, L);
+}
+// ... and code = clamp(rne(y / scale), -L, L), true IEEE division.
+__device__ __forceinline__ int32_t sym_code_div(float y, float scale, float L) {
+  return static_cast<int32_t>(fminf(fmaxf(rintf(__fdiv_rn(y, scale)), -L), L));
 }
 
 // code = clamp(rne(y / scale) + zero, 0, 15), with y / scale taken as y * fp32(1/scale).

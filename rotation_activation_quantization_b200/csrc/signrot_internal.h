@@ -48,8 +48,10 @@ struct RotateArgs {
   // quantized path -- q != null
   uint8_t* q;
   float* scale;
-  float* zero;
-  float clip;
+  float* zero;  // asymmetric grid only
+  float clip;   // asymmetric grid only
+  int32_t bits = 4;  // 4: two codes per byte; 8: one per byte
+  bool sym = false;  // symmetric grid (codes -L..L, no zero-point) instead of the asymmetric one
   float inv_sqrt_n;  // fp32(1 / sqrt(n))
 };
 

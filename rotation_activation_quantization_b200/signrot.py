@@ -31,6 +31,9 @@ _SIGNATURES = {
     "signrot_rotate_outlier": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_p],
     "signrot_rotate_quant_outlier": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_i32, _c_f,
                                      _c_p, _c_p, _c_p, _c_p],
+    "signrot_rotate_quant_sym": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_i32, _c_p, _c_p, _c_p],
+    "signrot_rotate_quant_sym_outlier": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_i32, _c_p,
+                                         _c_p, _c_p],
     "signrot_device_error": [_c_p, _c_i32],
     "signrot_rotate_quant_host": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_f,
                                   _c_p, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p],
@@ -196,16 +199,17 @@ def rotate(x: torch.Tensor, d: torch.Tensor, s: torch.Tensor | None = None,
 def rotate_quant(x: torch.Tensor, d: torch.Tensor, s: torch.Tensor | None = None, bits: int = 4,
                  clip: float = 1.0, q: torch.Tensor | None = None, scale: torch.Tensor | None = None,
                  zero: torch.Tensor | None = None, stream=None):
-    """The fused path: returns (q uint8 [T, n/2], scale f32 [T], zero f32 [T])."""
+    """The fused path: returns (q uint8 [T, n/2] (bits 4) or [T, n] (bits 8), scale f32 [T], zero f32 [T])."""
     T, n, ld = _rows(x)
     dev = x.device
     _need(d, dev, torch.int8, n, "d")
     if s is not None:
         _need(s, dev, torch.int8, n, "s")
-    q = torch.empty((T, n // 2), dtype=torch.uint8, device=dev) if q is None else q
+    qn = _q_row_bytes(n, bits)
+    q = torch.empty((T, qn), dtype=torch.uint8, device=dev) if q is None else q
     scale = torch.empty(T, dtype=torch.float32, device=dev) if scale is None else scale
     zero = torch.empty(T, dtype=torch.float32, device=dev) if zero is None else zero
-    _need(q, dev, torch.uint8, T * (n // 2), "q")
+    _need(q, dev, torch.uint8, T * qn, "q")
     _need(scale, dev, torch.float32, T, "scale")
     _need(zero, dev, torch.float32, T, "zero")
     with torch.cuda.device(dev):
@@ -243,10 +247,11 @@ def rotate_quant_outlier(x: torch.Tensor, d: torch.Tensor, k: torch.Tensor, xk: 
     _need(d, dev, torch.int8, n, "d")
     _need(k, dev, torch.int32, 1, "k")
     _need(xk, dev, torch.float32, 1, "xk")
-    q = torch.empty((T, n // 2), dtype=torch.uint8, device=dev) if q is None else q
+    qn = _q_row_bytes(n, bits)
+    q = torch.empty((T, qn), dtype=torch.uint8, device=dev) if q is None else q
     scale = torch.empty(T, dtype=torch.float32, device=dev) if scale is None else scale
     zero = torch.empty(T, dtype=torch.float32, device=dev) if zero is None else zero
-    _need(q, dev, torch.uint8, T * (n // 2), "q")
+    _need(q, dev, torch.uint8, T * qn, "q")
     _need(scale, dev, torch.float32, T, "scale")
     _need(zero, dev, torch.float32, T, "zero")
     with torch.cuda.device(dev):
@@ -255,6 +260,51 @@ def rotate_quant_outlier(x: torch.Tensor, d: torch.Tensor, k: torch.Tensor, xk: 
                                                 _stream(dev, stream))
     _check("signrot_rotate_quant_outlier", st)
     return q, scale, zero
+
+
+def _q_row_bytes(n: int, bits: int) -> int:
+    return n if bits == 8 else n // 2
+
+
+def rotate_quant_sym(x: torch.Tensor, d: torch.Tensor, s: torch.Tensor | None = None, bits: int = 4,
+                     q: torch.Tensor | None = None, scale: torch.Tensor | None = None, stream=None):
+    """Symmetric grid (codes -L..L, no zero-point): (q [T, n/2] two's-complement nibbles for bits 4,
+    or int8 [T, n] for bits 8, scale f32 [T])."""
+    T, n, ld = _rows(x)
+    dev = x.device
+    _need(d, dev, torch.int8, n, "d")
+    if s is not None:
+        _need(s, dev, torch.int8, n, "s")
+    qn = _q_row_bytes(n, bits)
+    q = torch.empty((T, qn), dtype=torch.int8 if bits == 8 else torch.uint8, device=dev) if q is None else q
+    scale = torch.empty(T, dtype=torch.float32, device=dev) if scale is None else scale
+    _need(q, dev, q.dtype, T * qn, "q")
+    _need(scale, dev, torch.float32, T, "scale")
+    with torch.cuda.device(dev):
+        st = lib().signrot_rotate_quant_sym(_ptr(x), _dtype_code(x), T, n, ld, _ptr(d), _ptr(s), int(bits),
+                                            _ptr(q), _ptr(scale), _stream(dev, stream))
+    _check("signrot_rotate_quant_sym", st)
+    return q, scale
+
+
+def rotate_quant_sym_outlier(x: torch.Tensor, d: torch.Tensor, k: torch.Tensor, xk: torch.Tensor, bits: int = 4,
+                             q: torch.Tensor | None = None, scale: torch.Tensor | None = None, stream=None):
+    """Symmetric grid with the sign vector folded in from (k, x_k): (q, scale)."""
+    T, n, ld = _rows(x)
+    dev = x.device
+    _need(d, dev, torch.int8, n, "d")
+    _need(k, dev, torch.int32, 1, "k")
+    _need(xk, dev, torch.float32, 1, "xk")
+    qn = _q_row_bytes(n, bits)
+    q = torch.empty((T, qn), dtype=torch.int8 if bits == 8 else torch.uint8, device=dev) if q is None else q
+    scale = torch.empty(T, dtype=torch.float32, device=dev) if scale is None else scale
+    _need(q, dev, q.dtype, T * qn, "q")
+    _need(scale, dev, torch.float32, T, "scale")
+    with torch.cuda.device(dev):
+        st = lib().signrot_rotate_quant_sym_outlier(_ptr(x), _dtype_code(x), T, n, ld, _ptr(d), _ptr(k), _ptr(xk),
+                                                    int(bits), _ptr(q), _ptr(scale), _stream(dev, stream))
+    _check("signrot_rotate_quant_sym_outlier", st)
+    return q, scale
 
 
 def device_error(clear: bool = True) -> int:

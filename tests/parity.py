@@ -62,17 +62,47 @@ def check_rotation(y_gpu: np.ndarray, y_ref: np.ndarray) -> dict:
     return {"rel_l2_max": float(rel.max()) if rel.size else 0.0, "max_abs": mx}
 
 
-def check_quant(q_gpu: np.ndarray, scale_gpu: np.ndarray, zero_gpu: np.ndarray, y_ref: np.ndarray,
-                clip: float = 1.0, x64: np.ndarray | None = None, strict: bool = True) -> dict:
+def decode_codes(q: np.ndarray, T: int, n: int, bits: int = 4, sym: bool = False) -> np.ndarray:
+    """Unpack the library's code layout to one int32 code per element: bits 4 -> two per byte
+    (element 2i in the low nibble; two's complement nibbles on the symmetric grid), bits 8 -> one
+    per byte (int8 on the symmetric grid)."""
+    q = np.asarray(q)
+    if bits == 8:
+        flat = q.reshape(T, n)
+        return flat.view(np.int8).astype(np.int32) if sym else flat.view(np.uint8).astype(np.int32)
+    nib = o.unpack_nibbles(q.view(np.uint8).reshape(T, n // 2)).astype(np.int32)
+    return ((nib ^ 8) - 8) if sym else nib
+
+
+def check_quant(q_gpu: np.ndarray, scale_gpu: np.ndarray, zero_gpu: np.ndarray | None, y_ref: np.ndarray,
+                clip: float = 1.0, x64: np.ndarray | None = None, strict: bool = True, bits: int = 4,
+                sym: bool = False) -> dict:
+    """Codes, scale and zero-point against the oracle's grid: asymmetric (codes 0 .. 2^bits - 1,
+    fp32 zero-point) or, with sym, symmetric (codes -L .. L, L = 2^(bits-1) - 1, no zero-point)."""
     T, n = y_ref.shape
-    codes_ref, scale_ref, zero_ref = o.quantize_asym(y_ref, clip=clip)
-    vpre, zpre = o.asym_preround(y_ref, clip=clip)
-    codes_gpu = o.unpack_nibbles(np.asarray(q_gpu, dtype=np.uint8).reshape(T, n // 2))
-    scale_gpu = np.asarray(scale_gpu, dtype=np.float32)
-    zero_gpu = np.asarray(zero_gpu, dtype=np.float32)
     y32 = y_ref.astype(np.float32)
-    lo_c = y32.min(axis=1).astype(np.float64) * clip
-    hi_c = y32.max(axis=1).astype(np.float64) * clip
+    if sym:
+        L = 2 ** (bits - 1) - 1
+        codes_ref, scale_ref = o.quantize_sym(y_ref, bits=bits)
+        codes_ref = codes_ref.astype(np.int32)
+        zero_ref = np.zeros(T, dtype=np.float32)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            vpre = y32 / scale_ref[:, None]
+        zpre = np.zeros(T, dtype=np.float32)
+        code_min, code_max = -L, L
+        lo_c = -np.abs(y32).max(axis=1).astype(np.float64)
+        hi_c = -lo_c
+        zero_gpu = np.zeros(T, dtype=np.float32)
+    else:
+        codes_ref, scale_ref, zero_ref = o.quantize_asym(y_ref, bits=bits, clip=clip)
+        codes_ref = codes_ref.astype(np.int32)
+        vpre, zpre = o.asym_preround(y_ref, bits=bits, clip=clip)
+        code_min, code_max = 0, 2 ** bits - 1
+        lo_c = y32.min(axis=1).astype(np.float64) * clip
+        hi_c = y32.max(axis=1).astype(np.float64) * clip
+        zero_gpu = np.asarray(zero_gpu, dtype=np.float32)
+    codes_gpu = decode_codes(q_gpu, T, n, bits, sym)
+    scale_gpu = np.asarray(scale_gpu, dtype=np.float32)
     rng = np.maximum(hi_c - lo_c, 1e-30)
 
     if strict:
@@ -101,10 +131,10 @@ def check_quant(q_gpu: np.ndarray, scale_gpu: np.ndarray, zero_gpu: np.ndarray, 
     shifted = np.flatnonzero(zdiff != 0)
     for t in shifted:  # the other side of a zero-point tie: redo the codes with the GPU's zero
         v = np.rint(y32[t] / scale_ref[t]) + zero_gpu[t]
-        codes_ref[t] = np.clip(v, 0, 15).astype(np.uint8)
+        codes_ref[t] = np.clip(v, code_min, code_max).astype(np.int32)
         vpre[t] = y32[t] / scale_ref[t] + zero_gpu[t]
 
-    diff = codes_gpu.astype(np.int32) - codes_ref.astype(np.int32)
+    diff = codes_gpu - codes_ref
     mism = diff != 0
     window = w_code[:, None]
     tie = _half_dist(vpre.astype(np.float64)) < window
@@ -121,8 +151,8 @@ def check_quant(q_gpu: np.ndarray, scale_gpu: np.ndarray, zero_gpu: np.ndarray, 
     assert n_well <= allowed, f"{n_well} tie mismatches on well-conditioned tokens > {allowed}"
     if not strict:
         deq = (codes_gpu.astype(np.float64) - zero_gpu[:, None]) * scale_gpu[:, None].astype(np.float64)
-        lo_g = (0 - zero_gpu.astype(np.float64)) * scale_gpu
-        hi_g = (15 - zero_gpu.astype(np.float64)) * scale_gpu
+        lo_g = (code_min - zero_gpu.astype(np.float64)) * scale_gpu
+        hi_g = (code_max - zero_gpu.astype(np.float64)) * scale_gpu
         yc = np.clip(y_ref, lo_g[:, None], hi_g[:, None])
         err = np.abs(deq - yc)
         lim = scale_gpu[:, None] * 0.5 * (1 + 1e-5) + delta[:, None] + 1e-30

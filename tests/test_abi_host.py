@@ -78,7 +78,8 @@ def test_validation_codes_without_cuda(binding):
     assert _rq(lib, n=1000) == binding.ERR_UNSUPPORTED_N
     assert _rq(lib, n=28 * 2048) == binding.ERR_UNSUPPORTED_N
     assert _rq(lib, n=1) == binding.ERR_UNSUPPORTED_N
-    assert _rq(lib, bits=8) == binding.ERR_UNSUPPORTED
+    assert _rq(lib, bits=5) == binding.ERR_UNSUPPORTED
+    assert _rq(lib, bits=2) == binding.ERR_UNSUPPORTED
     assert _rq(lib, clip=0.0) == binding.ERR_UNSUPPORTED
     assert _rq(lib, clip=1.5) == binding.ERR_UNSUPPORTED
     assert _rq(lib, dtype=7) == binding.ERR_INVALID_ARG
@@ -91,7 +92,6 @@ def test_validation_codes_without_cuda(binding):
     assert _rq(lib, dtype=1, x=(1 << 20) + 2) == binding.ERR_ALIGNMENT
     assert _rq(lib, scale=(1 << 23) + 2) == binding.ERR_ALIGNMENT
     assert _rq(lib, T=0) == binding.OK  # a no-op, no CUDA call
-    assert b"only 4" in lib.signrot_last_error() or True
     assert lib.signrot_rotate(None, 0, 0, 1000, 1000, 1, None, None, 1000, None) == binding.ERR_UNSUPPORTED_N
     assert lib.signrot_rotate(1 << 20, 0, 2, 64, 64, None, None, 1 << 21, 64, None) == binding.ERR_INVALID_ARG
     assert lib.signrot_rotate(1 << 20, 0, 2, 64, 64, 1 << 22, None, 1 << 21, 32, None) == binding.ERR_INVALID_ARG
@@ -101,6 +101,14 @@ def test_validation_codes_without_cuda(binding):
     assert lib.signrot_calibrate(1 << 20, 0, 4, 64, 64, 0, (1 << 21) + 4, 0, 1 << 22, 1 << 23, None) == binding.ERR_ALIGNMENT
     assert lib.signrot_calibrate(1 << 20, 0, 4, 64, 64, 0x7ffffffe, 1 << 21, 0, 1 << 22, 1 << 23, None) == binding.ERR_INVALID_ARG
     assert lib.signrot_get_h28(None) == binding.ERR_INVALID_ARG
+    # the symmetric grid: bits 4 or 8, scale required, no zero-point pointer
+    sym = lib.signrot_rotate_quant_sym
+    assert sym(1 << 20, 0, 4, 1024, 1024, 1 << 21, None, 6, 1 << 22, 1 << 23, None) == binding.ERR_UNSUPPORTED
+    assert sym(1 << 20, 0, 4, 1024, 1024, 1 << 21, None, 4, 1 << 22, None, None) == binding.ERR_INVALID_ARG
+    assert sym(1 << 20, 0, 4, 1000, 1000, 1 << 21, None, 4, 1 << 22, 1 << 23, None) == binding.ERR_UNSUPPORTED_N
+    assert sym(1 << 20, 0, 0, 1024, 1024, 1 << 21, None, 8, 1 << 22, 1 << 23, None) == binding.OK
+    symo = lib.signrot_rotate_quant_sym_outlier
+    assert symo(1 << 20, 0, 4, 1024, 1024, 1 << 21, None, 1 << 24, 4, 1 << 22, 1 << 23, None) == binding.ERR_INVALID_ARG
 
 
 def test_error_messages(binding):
