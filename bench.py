@@ -48,6 +48,8 @@ def parse(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quant", choices=["asym4", "asym8", "sym4", "sym8"], default="asym4",
+                    help="grid of the timed kernel: asymmetric INT4 (the metric's), INT8, or symmetric")
     return ap.parse_args(argv)
 
 
@@ -56,9 +58,11 @@ def workload(args) -> syn.Workload:
     return w.with_T(args.tokens) if args.tokens else w
 
 
-def bytes_per_token(w: syn.Workload) -> int:
-    """Algorithmic HBM bytes per token: activations in, packed INT4 out, fp32 scale + zero."""
-    return w.in_bytes * w.n + w.n // 2 + 8
+def bytes_per_token(w: syn.Workload, quant: str = "asym4") -> int:
+    """Algorithmic HBM bytes per token: activations in, codes out (packed two per byte for 4 bits,
+    one per byte for 8), fp32 scale (+ fp32 zero-point on the asymmetric grid)."""
+    bits = 8 if quant.endswith("8") else 4
+    return w.in_bytes * w.n + w.n * bits // 8 + (4 if quant.startswith("sym") else 8)
 
 
 def measured_peaks() -> dict:
@@ -270,12 +274,17 @@ def run_ours(args) -> int:
     calib_ms = c0.elapsed_time(c1)
     del xc
 
-    q = torch.empty((T, n // 2), dtype=torch.uint8, device=dev)
+    bits = 8 if args.quant.endswith("8") else 4
+    sym = args.quant.startswith("sym")
+    q = torch.empty((T, n * bits // 8), dtype=torch.int8 if (sym and bits == 8) else torch.uint8, device=dev)
     scale = torch.empty(T, dtype=torch.float32, device=dev)
     zero = torch.empty(T, dtype=torch.float32, device=dev)
 
     def step():
-        sr.rotate_quant_outlier(x, d, k, xk, q=q, scale=scale, zero=zero)
+        if sym:
+            sr.rotate_quant_sym_outlier(x, d, k, xk, bits=bits, q=q, scale=scale)
+        else:
+            sr.rotate_quant_outlier(x, d, k, xk, bits=bits, q=q, scale=scale, zero=zero)
 
     for _ in range(args.warmup):
         step()
@@ -331,16 +340,16 @@ def run_ours(args) -> int:
     if world > 1:
         dist.barrier()
     h2d = x.numel() * x.element_size()
-    d2h = q.numel() + 4 * scale.numel() + 4 * zero.numel()
+    d2h = qh.numel() + 4 * sh.numel() + 4 * zh.numel()
 
     if rank == 0:
-        bpt = bytes_per_token(w)
+        bpt = bytes_per_token(w, args.quant)
         bytes_per_launch = bpt * T
         avg_launch_ms = region_ms / K  # the fused kernel is the only launch in the region
         achieved = bytes_per_launch / (avg_launch_ms * 1e-3) / 1e9
         peaks = measured_peaks()
         digest = kernel_sources_digest()
-        traffic = recorded_traffic(w, digest)
+        traffic = recorded_traffic(w, digest) if args.quant == "asym4" else None
         value = sharding.aggregate_rate(world * T * K, region_ms_max * 1e-3)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -348,7 +357,11 @@ def run_ours(args) -> int:
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {
                 "workload": w.name, "n": n, "tokens_per_gpu": T, "global_tokens": world * T,
-                "input_dtype": w.dtype, "output": "INT4 packed [T, n/2] + fp32 scale/zero [T]",
+                "input_dtype": w.dtype, "quant": args.quant,
+                "output": {"asym4": "INT4 packed [T, n/2] + fp32 scale/zero [T]",
+                           "asym8": "INT8 [T, n] + fp32 scale/zero [T]",
+                           "sym4": "signed INT4 packed [T, n/2] + fp32 scale [T]",
+                           "sym8": "int8 [T, n] + fp32 scale [T]"}[args.quant],
                 "parallelism": f"token-sharded x{world} (no collective)",
                 "l2": f"inputs larger than L2 ({bytes_per_launch / 1e6:.1f} MB per step vs "
                       f"{L2_BYTES / 1e6:.0f} MB), no flush",
@@ -359,12 +372,14 @@ def run_ours(args) -> int:
                 "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                 "peak_source": peaks["source"], "bytes_per_token": bpt,
-                "kernel": "signrot_rotate_quant", "kernel_sources": digest,
+                "kernel": "signrot_rotate_quant" if not sym else "signrot_rotate_quant_sym",
+                "kernel_sources": digest,
                 "launch_ms_mean": avg_launch_ms,
             },
             "e2e": {"value": world * T * E / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms / E, "steps": E},
+                    "ms_per_step": e2e_ms / E, "steps": E,
+                    "call": "signrot_rotate_quant_host (asymmetric INT4 grid)"},
             "gpu_launches": int(launches),
             "calibration": {"tokens": int(xc_np.shape[0]), "ms": calib_ms,
                             "gbs": xc_np.shape[0] * n * w.in_bytes / (calib_ms * 1e-3) / 1e9},
