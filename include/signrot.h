@@ -19,10 +19,15 @@
  * "The flip alone does nothing for a symmetric quantizer" (asymmetric zero-point) and "Worked
  * example" (steps are range/15, no clipping).
  *
- * H = H_F kron H_M with n = F * M, F in {1, 28}, M = 2^m, channel j = a * M + b. H_M is
- * Sylvester's (H_M[b][e] = (-1)^popcount(b & e)); H_28 is Paley's construction I over
- * GF(27) = GF(3)[t]/(t^3 + 2t + 1) (row 0 all +1, column 0 = (1, -1, ..., -1), see
- * signrot_get_h28). Supported n: 2^m for 1 <= m <= 15, and 28 * 2^m for 0 <= m <= 10.
+ * H = H_F kron H_M with n = F * M, F in {1, 28, 344}, M = 2^m, channel j = a * M + b. H_M is
+ * Sylvester's (H_M[b][e] = (-1)^popcount(b & e)); H_28 and H_344 are Paley's construction I
+ * over GF(27) = GF(3)[t]/(t^3 + 2t + 1) and GF(343) = GF(7)[t]/(t^3 + t + 1): row 0 all +1,
+ * column 0 = (1, -1, ..., -1), H[1+e][1+f] = [e == f] + chi(e - f) with field element
+ * e = c0 + p c1 + p^2 c2 and chi the quadratic character (see signrot_get_h28/_h344).
+ * Supported n: 2^m for 1 <= m <= 15, 28 * 2^m for 0 <= m <= 10, and 344 * 2^m for
+ * 0 <= m <= 5 (n = 11008 = 344 * 32 is LLaMA-2-7B's MLP width, the example in the
+ * explainer's paragraph "Here is how it breaks"). F = 344 runs on the generic kernel (fp64
+ * accumulation on the CUDA cores).
  *
  * Conventions shared by every call:
  *   - Every call returns a signrot_status; nothing is thrown across the ABI.
@@ -48,7 +53,7 @@ extern "C" {
 typedef int32_t signrot_status;
 #define SIGNROT_OK 0
 #define SIGNROT_ERR_INVALID_ARG 1   /* null pointer, negative size, ld < n, bad dtype, ... */
-#define SIGNROT_ERR_UNSUPPORTED_N 2 /* n not of the form 2^m or 28 * 2^m (see above)      */
+#define SIGNROT_ERR_UNSUPPORTED_N 2 /* n not of a supported form (see above)              */
 #define SIGNROT_ERR_ALIGNMENT 3     /* pointer not aligned to its element type            */
 #define SIGNROT_ERR_CUDA 4          /* a CUDA runtime call failed; see signrot_last_error */
 #define SIGNROT_ERR_UNSUPPORTED 5   /* e.g. bits != 4, clip outside (0, 1]                 */
@@ -212,6 +217,10 @@ signrot_status signrot_device_error(int32_t* code, int32_t clear);
 
 /* Host: writes H_28 (Paley, GF(27), the orientation described above) row-major into out[784]. */
 signrot_status signrot_get_h28(int8_t* out);
+
+/* Host: writes H_344 (Paley, GF(343), the orientation described above) row-major into
+ * out[344 * 344]. */
+signrot_status signrot_get_h344(int8_t* out);
 
 /* 1 if n is a supported row length, else 0. */
 int32_t signrot_supported_n(int32_t n);

@@ -92,9 +92,10 @@ __global__ void __launch_bounds__(1024) calib_argmax_kernel(const unsigned long 
   }
 }
 
-// s_j = +1 if H[j][k] * D_k * x_k >= 0 else -1, H[(a,b),(c,e)] = H_28[a][c] (-1)^popcount(b & e).
+// s_j = +1 if H[j][k] * D_k * x_k >= 0 else -1, H[(a,b),(c,e)] = H_F[a][c] (-1)^popcount(b & e).
 __global__ void build_sign_kernel(Shape sh, const int32_t* __restrict__ kp, const float* __restrict__ xkp,
-                                  const int8_t* __restrict__ d, int8_t* __restrict__ s, H28Masks h) {
+                                  const int8_t* __restrict__ d, int8_t* __restrict__ s, H28Masks h,
+                                  GF343Squares sq) {
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= sh.n) return;
   const int k = *kp;
@@ -108,6 +109,7 @@ __global__ void build_sign_kernel(Shape sh, const int32_t* __restrict__ kp, cons
   const int c = k >> sh.logM, e = k & M1;
   int neg = __popc(b & e) & 1;
   if (sh.F == 28) neg ^= static_cast<int>((h.row[a] >> c) & 1u);
+  if (sh.F == 344) neg ^= h344_neg(sq, a, c);
   const float hv = neg ? -1.f : 1.f;
   const float v = hv * static_cast<float>(d[k]) * xk;  // exact: +/-1 factors
   s[j] = v >= 0.f ? int8_t(1) : int8_t(-1);
@@ -137,10 +139,10 @@ cudaError_t launch_calibrate_argmax(const unsigned long long* ws, int32_t n, int
 }
 
 cudaError_t launch_build_sign(Shape shape, const int32_t* k, const float* xk, const int8_t* d,
-                              int8_t* s_out, const H28Masks& h, cudaStream_t st) {
+                              int8_t* s_out, const H28Masks& h, const GF343Squares& sq, cudaStream_t st) {
   const int threads = 256;
   const int grid = (shape.n + threads - 1) / threads;
-  build_sign_kernel<<<grid, threads, 0, st>>>(shape, k, xk, d, s_out, h);
+  build_sign_kernel<<<grid, threads, 0, st>>>(shape, k, xk, d, s_out, h, sq);
   count_launch();
   return cudaGetLastError();
 }

@@ -5,7 +5,7 @@
 // Per row (SignRot explainer, "The standard fix is rotation" and "SignRot asks one crowd to walk
 // across the hall"; abstract: fast Walsh-Hadamard transform):
 //   1. x' = D (.) x                 (exact sign flips)
-//   2. H_28 across the stride-M axis (dense 28 x 28 block, F = 28 only)
+//   2. H_F across the stride-M axis (dense 28 x 28 or 344 x 344 block, F > 1 only)
 //   3. FWHT of length M along the contiguous axis, radix-2 stages
 //   4. y = s (.) w / sqrt(n), rounded once to fp32
 //   5. check path: store y; quantized path: row min/max, the asymmetric (scale, zero) or symmetric
@@ -30,7 +30,8 @@ __device__ __forceinline__ Acc neg_if(Acc v, bool neg) {
 }
 
 template <typename Tin, typename Acc, bool kQuant>
-__global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, H28Masks h, double sqrt_n) {
+__global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, H28Masks h, GF343Squares sq,
+                                                                  double sqrt_n) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Acc* buf = reinterpret_cast<Acc*>(smem_raw);
   float* ybuf = reinterpret_cast<float*>(smem_raw);  // fp32 y, aliases buf after step 4
@@ -38,6 +39,21 @@ __global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, 
   const int n = a.shape.n;
   const int logM = a.shape.logM;
   const int M = 1 << logM;
+  const bool f344 = a.shape.F == 344;
+  // F = 344: the mixed row goes to a second buffer (the block is too large to hold a column in
+  // registers), and the block's sign masks sit after it: bit c % 32 of hm[r * 11 + c / 32] is
+  // set iff H_344[r][c] == -1.
+  Acc* mixed = f344 ? buf + n : buf;
+  uint32_t* hm = reinterpret_cast<uint32_t*>(smem_raw + 2 * static_cast<size_t>(n) * sizeof(Acc));
+  if (f344) {
+    for (int w = threadIdx.x; w < 344 * 11; w += blockDim.x) {
+      const int r = w / 11, c0 = (w % 11) * 32;
+      uint32_t bits = 0;
+      for (int cc = 0; cc < 32 && c0 + cc < 344; ++cc) bits |= static_cast<uint32_t>(h344_neg(sq, r, c0 + cc)) << cc;
+      hm[w] = bits;
+    }
+    __syncthreads();
+  }
   const Tin* __restrict__ x = static_cast<const Tin*>(a.x);
   // sign vector from the outlier channel: s_j = sgn(H[j,k] D_k x_k), +1 everywhere if x_k = 0
   bool pattern = false;
@@ -73,6 +89,28 @@ __global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, 
         }
       }
       __syncthreads();
+    } else if (f344) {
+      // eight output rows of one column per work item; c ascending, a fixed summation order
+      for (int item = threadIdx.x; item < M * 43; item += blockDim.x) {
+        const int b = item % M, r0 = (item / M) * 8;
+        Acc acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0;
+        for (int w = 0; w < 11; ++w) {
+          uint32_t m[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m[i] = hm[(r0 + i) * 11 + w];
+          const int cn = w < 10 ? 32 : 344 - 320;
+          for (int cc = 0; cc < cn; ++cc) {
+            const Acc v = buf[(w * 32 + cc) * M + b];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] += neg_if(v, (m[i] >> cc) & 1u);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mixed[(r0 + i) * M + b] = acc[i];
+      }
+      __syncthreads();
     }
 
     for (int hs = 1; hs < M; hs <<= 1) {
@@ -80,7 +118,7 @@ __global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, 
         const int row = p >> (logM - 1);
         const int r = p & ((M >> 1) - 1);
         const int i = ((r & ~(hs - 1)) << 1) | (r & (hs - 1));
-        Acc* base = buf + row * M;
+        Acc* base = mixed + row * M;
         const Acc u = base[i], v = base[i + hs];
         base[i] = u + v;
         base[i + hs] = u - v;
@@ -102,10 +140,11 @@ __global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, 
           if (pattern) {
             neg = ((__popc((j & (M - 1)) & e_k) & 1) ^ sig_neg) != 0;
             if (a.shape.F == 28) neg ^= ((h.row[j >> logM] >> c_k) & 1u) != 0;
+            if (f344) neg ^= ((hm[(j >> logM) * 11 + (c_k >> 5)] >> (c_k & 31)) & 1u) != 0;
           } else {
             neg = a.s != nullptr && a.s[j] < 0;
           }
-          const Acc w = neg_if(buf[j], neg);
+          const Acc w = neg_if(mixed[j], neg);
           yv[e] = sizeof(Acc) == 8 ? static_cast<float>(static_cast<double>(w) / sqrt_n)
                                    : static_cast<float>(w) * a.inv_sqrt_n;
         }
@@ -168,8 +207,9 @@ __global__ void __launch_bounds__(kThreads) rotate_generic_kernel(RotateArgs a, 
 }
 
 template <typename Tin, typename Acc, bool kQuant>
-cudaError_t launch_typed(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(a.shape.n) * sizeof(Acc);
+cudaError_t launch_typed(const RotateArgs& a, const H28Masks& h, const GF343Squares& sq, cudaStream_t st) {
+  const size_t row = static_cast<size_t>(a.shape.n) * sizeof(Acc);
+  const size_t smem = a.shape.F == 344 ? 2 * row + 344 * 11 * sizeof(uint32_t) : row;
   auto kern = rotate_generic_kernel<Tin, Acc, kQuant>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -181,23 +221,25 @@ cudaError_t launch_typed(const RotateArgs& a, const H28Masks& h, cudaStream_t st
     return e;
   const int64_t cap = static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1);
   const int grid = static_cast<int>(a.T < cap ? a.T : cap);
-  kern<<<grid, kThreads, smem, st>>>(a, h, sqrt(static_cast<double>(a.shape.n)));
+  kern<<<grid, kThreads, smem, st>>>(a, h, sq, sqrt(static_cast<double>(a.shape.n)));
   count_launch();
   return cudaGetLastError();
 }
 
 template <typename Tin, typename Acc>
-cudaError_t launch_acc(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
-  return a.q != nullptr ? launch_typed<Tin, Acc, true>(a, h, st) : launch_typed<Tin, Acc, false>(a, h, st);
+cudaError_t launch_acc(const RotateArgs& a, const H28Masks& h, const GF343Squares& sq, cudaStream_t st) {
+  return a.q != nullptr ? launch_typed<Tin, Acc, true>(a, h, sq, st) : launch_typed<Tin, Acc, false>(a, h, sq, st);
 }
 
 }  // namespace
 
-cudaError_t launch_rotate_generic(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
-  const bool wide = a.shape.n <= 28672;  // fp64 row fits in shared memory
+cudaError_t launch_rotate_generic(const RotateArgs& a, const H28Masks& h, const GF343Squares& sq,
+                                  cudaStream_t st) {
+  // fp64 row (two of them and the sign masks for F = 344, n <= 11008) fits in shared memory
+  const bool wide = a.shape.n <= 28672;
   if (a.dtype == kBF16)
-    return wide ? launch_acc<uint16_t, double>(a, h, st) : launch_acc<uint16_t, float>(a, h, st);
-  return wide ? launch_acc<float, double>(a, h, st) : launch_acc<float, float>(a, h, st);
+    return wide ? launch_acc<uint16_t, double>(a, h, sq, st) : launch_acc<uint16_t, float>(a, h, sq, st);
+  return wide ? launch_acc<float, double>(a, h, sq, st) : launch_acc<float, float>(a, h, sq, st);
 }
 
 }  // namespace signrot

@@ -1272,6 +1272,7 @@ cudaError_t dispatch_stream(const TcParams& p, bool vec_sign, int mode, cudaStre
 
 cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
   if (a.dtype != kBF16 || a.T <= 0 || a.T > 0x7fffffff) return cudaErrorNotSupported;
+  if (a.shape.F != 1 && a.shape.F != 28) return cudaErrorNotSupported;
   const bool f28 = a.shape.F == 28;
   const int ncol = f28 ? (1 << a.shape.logM) / 4 : a.shape.n / 128;
   if (ncol != 64 && ncol != 128 && ncol != 256) return cudaErrorNotSupported;

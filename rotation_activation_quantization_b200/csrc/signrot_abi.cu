@@ -52,8 +52,15 @@ bool factor_n(int32_t n, signrot::Shape* sh) {
     *sh = {n, 28, lg(n / 28)};
     return true;
   }
+  if (n % 344 == 0 && pow2(n / 344) && n / 344 <= 32) {
+    *sh = {n, 344, lg(n / 344)};
+    return true;
+  }
   return false;
 }
+
+#define SIGNROT_N_FORMS "2^m (1<=m<=15), 28*2^m (0<=m<=10) or 344*2^m (0<=m<=5)"
+
 
 struct H28State {
   int8_t h[28][28];
@@ -73,6 +80,13 @@ const H28State& h28_state() {
     }
   });
   return st;
+}
+
+const signrot::GF343Squares& gf343_state() {
+  static signrot::GF343Squares sq;
+  static std::once_flag once;
+  std::call_once(once, [] { sq = signrot::gf343_squares(); });
+  return sq;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -112,7 +126,7 @@ signrot_status check_rows(const void* x, int32_t dtype, int64_t T, int32_t n, in
     return fail(SIGNROT_ERR_INVALID_ARG, "dtype %d is neither SIGNROT_BF16 nor SIGNROT_F32", dtype);
   if (T < 0) return fail(SIGNROT_ERR_INVALID_ARG, "T = %lld < 0", static_cast<long long>(T));
   if (!factor_n(n, sh))
-    return fail(SIGNROT_ERR_UNSUPPORTED_N, "n = %d is not 2^m (1<=m<=15) or 28*2^m (0<=m<=10)", n);
+    return fail(SIGNROT_ERR_UNSUPPORTED_N, "n = %d is not " SIGNROT_N_FORMS, n);
   if (ld < n) return fail(SIGNROT_ERR_INVALID_ARG, "ld = %lld < n = %d", static_cast<long long>(ld), n);
   if (T > 0 && x == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "x is NULL");
   if (!aligned(x, dtype == SIGNROT_BF16 ? 2 : 4))
@@ -126,7 +140,7 @@ signrot_status run_rotate(signrot::RotateArgs& a, cudaStream_t st) {
   cudaError_t e = signrot::launch_rotate_fast(a, h, st);
   if (e == cudaErrorNotSupported) {
     (void)cudaGetLastError();
-    e = signrot::launch_rotate_generic(a, h, st);
+    e = signrot::launch_rotate_generic(a, h, gf343_state(), st);
   }
   if (e != cudaSuccess) return cuda_fail(e, "rotate launch");
   return SIGNROT_OK;
@@ -233,11 +247,11 @@ signrot_status signrot_build_sign(int32_t n, const int32_t* k, const float* xk, 
   g_last_error[0] = '\0';
   signrot::Shape sh;
   if (!factor_n(n, &sh))
-    return fail(SIGNROT_ERR_UNSUPPORTED_N, "n = %d is not 2^m (1<=m<=15) or 28*2^m (0<=m<=10)", n);
+    return fail(SIGNROT_ERR_UNSUPPORTED_N, "n = %d is not " SIGNROT_N_FORMS, n);
   if (k == nullptr || xk == nullptr || d == nullptr || s_out == nullptr)
     return fail(SIGNROT_ERR_INVALID_ARG, "k, xk, d and s_out must be device pointers");
   if (!aligned(k, 4) || !aligned(xk, 4)) return fail(SIGNROT_ERR_ALIGNMENT, "k or xk misaligned");
-  cudaError_t e = signrot::launch_build_sign(sh, k, xk, d, s_out, h28_state().masks,
+  cudaError_t e = signrot::launch_build_sign(sh, k, xk, d, s_out, h28_state().masks, gf343_state(),
                                              static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "build_sign launch");
   return SIGNROT_OK;
@@ -384,6 +398,12 @@ signrot_status signrot_device_error(int32_t* code, int32_t clear) {
 signrot_status signrot_get_h28(int8_t* out) {
   if (out == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "out is NULL");
   std::memcpy(out, h28_state().h, 28 * 28);
+  return SIGNROT_OK;
+}
+
+signrot_status signrot_get_h344(int8_t* out) {
+  if (out == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "out is NULL");
+  signrot::paley_h344(out);
   return SIGNROT_OK;
 }
 

@@ -5,7 +5,23 @@
 
 #include <cuda_runtime.h>
 
+#include "signrot_internal.h"
+
 namespace signrot {
+
+// 1 iff H_344[i][j] == -1 (Paley construction I over GF(343), element e = c0 + 7 c1 + 49 c2):
+// row 0 is all +1, column 0 below it all -1, and H[1+e][1+f] = [e == f] + chi(e - f).
+__host__ __device__ __forceinline__ int h344_neg(const GF343Squares& sq, int i, int j) {
+  if (i == 0) return 0;
+  if (j == 0) return 1;
+  if (i == j) return 0;
+  const int e = i - 1, f = j - 1;
+  const int d0 = (e % 7 - f % 7 + 7) % 7;
+  const int d1 = ((e / 7) % 7 - (f / 7) % 7 + 7) % 7;
+  const int d2 = (e / 49 - f / 49 + 7) % 7;
+  const int d = d0 + 7 * d1 + 49 * d2;
+  return ((sq.bits[d >> 5] >> (d & 31)) & 1u) ? 0 : 1;
+}
 
 __device__ __forceinline__ float load_as_float(const uint16_t* p) {
   return __uint_as_float(static_cast<uint32_t>(*p) << 16);  // bf16 -> fp32 is exact

@@ -13,8 +13,9 @@ void count_launch(int n = 1);
 // Sets the message signrot_last_error returns on this host thread.
 void set_last_error(const char* msg);
 
-// Library-owned Paley H_28 (paley_gf27.cpp), row-major, entries +/-1.
+// Library-owned Paley matrices (paley.cpp), row-major, entries +/-1.
 void paley_h28(int8_t h[28][28]);
+void paley_h344(int8_t* h);  // [344 * 344]
 
 // H_28 as sign masks: bit c of row[a] is set iff H_28[a][c] == -1. Passed by value in kernel
 // parameters (constant bank), so no per-device state has to be initialised.
@@ -22,9 +23,17 @@ struct H28Masks {
   uint32_t row[28];
 };
 
+// The nonzero squares of GF(343) = GF(7)[t]/(t^3 + t + 1) (bit e set iff element e is one),
+// element e = c0 + 7 c1 + 49 c2. With them H_344[1+e][1+f] = -1 iff e != f and e - f (digitwise
+// mod 7) is a non-square; row 0 is all +1 and column 0 below it all -1. Passed by value.
+struct GF343Squares {
+  uint32_t bits[11];
+};
+GF343Squares gf343_squares();
+
 enum : int32_t { kBF16 = 0, kF32 = 1 };
 
-// n = F * 2^logM, F in {1, 28}.
+// n = F * 2^logM, F in {1, 28, 344}.
 struct Shape {
   int32_t n;
   int32_t F;
@@ -56,7 +65,8 @@ struct RotateArgs {
 };
 
 // Generic row kernel: any supported n, any element-aligned x. One CTA per row (grid-stride).
-cudaError_t launch_rotate_generic(const RotateArgs& a, const H28Masks& h, cudaStream_t st);
+cudaError_t launch_rotate_generic(const RotateArgs& a, const H28Masks& h, const GF343Squares& sq,
+                                  cudaStream_t st);
 
 // Fast fused kernels for the shapes they cover; return cudaErrorNotSupported when the shape or
 // the alignment is not theirs (the caller then uses the generic kernel).
@@ -78,6 +88,6 @@ cudaError_t launch_calibrate_fold(const CalibArgs& a, cudaStream_t st);
 cudaError_t launch_calibrate_argmax(const unsigned long long* ws, int32_t n, int32_t* k_out,
                                     float* xk_out, cudaStream_t st);
 cudaError_t launch_build_sign(Shape shape, const int32_t* k, const float* xk, const int8_t* d,
-                              int8_t* s_out, const H28Masks& h, cudaStream_t st);
+                              int8_t* s_out, const H28Masks& h, const GF343Squares& sq, cudaStream_t st);
 
 }  // namespace signrot

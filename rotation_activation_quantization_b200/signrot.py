@@ -39,6 +39,7 @@ _SIGNATURES = {
                                   _c_p, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p],
     "signrot_host_bytes_per_token": [_c_i32, _c_i32],
     "signrot_get_h28": [_c_p],
+    "signrot_get_h344": [_c_p],
     "signrot_supported_n": [_c_i32],
     "signrot_status_string": [_c_i32],
     "signrot_last_error": [],
@@ -128,6 +129,12 @@ def get_h28() -> np.ndarray:
     out = np.zeros(28 * 28, dtype=np.int8)
     _check("signrot_get_h28", lib().signrot_get_h28(out.ctypes.data))
     return out.reshape(28, 28)
+
+
+def get_h344() -> np.ndarray:
+    out = np.zeros(344 * 344, dtype=np.int8)
+    _check("signrot_get_h344", lib().signrot_get_h344(out.ctypes.data))
+    return out.reshape(344, 344)
 
 
 def calibrate(x: torch.Tensor, ws: torch.Tensor | None = None, accumulate: bool = False,

@@ -54,11 +54,21 @@ def test_library_h28_equals_oracle_h28(binding):
     assert (binding.get_h28() == o.paley_h28()).all()
 
 
+def test_library_h344_equals_oracle_h344(binding):
+    h = binding.get_h344()
+    assert (h == o.paley_h344()).all()
+    # and, apart from the oracle: a skew Hadamard matrix with the stated border
+    assert (h.astype(np.int64) @ h.T.astype(np.int64) == 344 * np.eye(344, dtype=np.int64)).all()
+    assert (h + h.T == 2 * np.eye(344, dtype=np.int8)).all()
+    assert (h[0] == 1).all() and (h[1:, 0] == -1).all()
+
+
 def test_supported_n_matches_oracle(binding):
-    for n in list(range(0, 200)) + [1024, 4096, 11008, 14336, 28672, 32768, 65536, 28 * 2048]:
+    for n in list(range(0, 400)) + [688, 1024, 4096, 5504, 11008, 14336, 22016, 28672, 32768, 65536,
+                                    28 * 2048]:
         try:
             F, M = o.factor_n(n)
-            expect = F in (1, 28) and (F * M <= 32768 if F == 1 else M <= 1024)
+            expect = (F == 1 and n <= 32768) or (F == 28 and M <= 1024) or (F == 344 and M <= 32)
         except ValueError:
             expect = False
         assert binding.supported_n(n) == expect, n
