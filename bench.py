@@ -50,6 +50,9 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quant", choices=["asym4", "asym8", "sym4", "sym8"], default="asym4",
                     help="grid of the timed kernel: asymmetric INT4 (the metric's), INT8, or symmetric")
+    ap.add_argument("--sweep", action="store_true",
+                    help="decode/prefill sweep at n = 14336 (T = 1 .. 32768, latency per call and GB/s, "
+                         "warm and after an L2 flush) and the 128 x 2048-token calibration pass; one GPU")
     return ap.parse_args(argv)
 
 
@@ -396,9 +399,141 @@ def run_ours(args) -> int:
     return 0
 
 
+def run_sweep(args) -> int:
+    """Decode/prefill sweep of the fused call and the calibration pass over 128 x 2048 tokens.
+
+    Rows: the first 8192 tokens of the sweep workload drawn on the host, tiled 4x on the device
+    for T = 32768; calibration: its first 8192 calibration rows tiled 32x (262144 tokens, 7.5 GB).
+    Tiling changes no work: every kernel here reads every row and does the same arithmetic on it.
+    """
+    import torch
+
+    from rotation_activation_quantization_b200 import signrot as sr
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    sr.lib()
+    w = syn.workload(5)
+    n, Tmax = w.n, max(syn.SWEEP_T)
+    base = 8192
+
+    def bf(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x = bf(syn.draw_tokens(w, 0, base)).repeat(Tmax // base, 1)
+    d = torch.from_numpy(syn.draw_d(w)).to(dev)
+    xc = bf(syn.draw_calibration(w, 0, base)).repeat(w.calib_T // base, 1)
+    stream = torch.cuda.current_stream(dev)
+    ws = torch.empty(n, dtype=torch.int64, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    peaks = measured_peaks()
+    bpt = bytes_per_token(w)
+
+    def timed(fn, reps, flush_l2):
+        times = []
+        for _ in range(reps):
+            if flush_l2:
+                flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            times.append(e0.elapsed_time(e1))
+        return float(np.median(times)), float(np.min(times))
+
+    # calibration: one call over all 262144 tokens, and 128 calls of 2048 continuing one another
+    def calib_once():
+        k, xk, _ = sr.calibrate(xc, ws=ws)
+        sr.build_sign(n, k, xk, d)
+
+    def calib_chunked():
+        for i in range(w.calib_T // 2048):
+            k, xk, _ = sr.calibrate(xc[i * 2048:(i + 1) * 2048], ws=ws, accumulate=i > 0, t_offset=i * 2048)
+        sr.build_sign(n, k, xk, d)
+
+    calib_once()
+    calib_chunked()
+    torch.cuda.synchronize(dev)
+    cal_bytes = w.calib_T * n * 2
+    one_med, one_min = timed(calib_once, 5, True)
+    ch_med, _ = timed(calib_chunked, 3, True)
+    k, xk, _ = sr.calibrate(xc, ws=ws)
+    del xc
+    torch.cuda.synchronize(dev)
+
+    q = torch.empty((Tmax, n // 2), dtype=torch.uint8, device=dev)
+    scale = torch.empty(Tmax, dtype=torch.float32, device=dev)
+    zero = torch.empty(Tmax, dtype=torch.float32, device=dev)
+    rows = []
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        for T in syn.SWEEP_T:
+            xs, qs, ss, zs = x[:T], q[:T], scale[:T], zero[:T]
+
+            def call():
+                sr.rotate_quant_outlier(xs, d, k, xk, q=qs, scale=ss, zero=zs)
+
+            for _ in range(max(3, args.warmup)):
+                call()
+            K = 200 if T <= 4096 else max(20, args.steps // 4)
+            torch.cuda.synchronize(dev)
+            l0 = sr.kernel_launches()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(K):
+                call()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            launches = sr.kernel_launches() - l0
+            warm_ms = e0.elapsed_time(e1) / K
+            cold_ms, _ = timed(call, 20, True)
+            rows.append({"T": T, "us_per_call_back_to_back": warm_ms * 1e3,
+                         "gbs_back_to_back": T * bpt / (warm_ms * 1e-3) / 1e9,
+                         "us_per_call_l2_flushed": cold_ms * 1e3,
+                         "gbs_l2_flushed": T * bpt / (cold_ms * 1e-3) / 1e9,
+                         "tokens_per_s_back_to_back": T / (warm_ms * 1e-3), "steps": K,
+                         "gpu_launches": int(launches)})
+    top = rows[-1]
+    achieved = top["gbs_back_to_back"]
+    line = {
+        "metric": METRIC, "value": top["tokens_per_s_back_to_back"], "unit": UNIT, "n_gpus": 1,
+        "steps": top["steps"], "warmup": max(3, args.warmup), "ms_per_step": top["us_per_call_back_to_back"] * 1e-3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (8192 drawn rows tiled to 32768; 8192 calibration rows tiled to 262144)",
+        "config": {"workload": w.name, "n": n, "sweep_T": list(syn.SWEEP_T), "input_dtype": w.dtype,
+                   "quant": "asym4",
+                   "l2": "back-to-back rows: inputs below 126 MB stay in L2 (T <= 4096); "
+                         "flushed rows: a 252 MB write before each timed call"},
+        "sweep": rows,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
+                     "bytes_per_token": bpt, "kernel": "signrot_rotate_quant (T = 32768)",
+                     "kernel_sources": kernel_sources_digest()},
+        "calibration": {
+            "tokens": w.calib_T, "bytes": cal_bytes,
+            "one_call_ms": one_med, "one_call_gbs": cal_bytes / (one_med * 1e-3) / 1e9,
+            "one_call_frac": cal_bytes / (one_med * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "one_call_ms_min": one_min,
+            "chunked_128x2048_ms": ch_med, "chunked_gbs": cal_bytes / (ch_med * 1e-3) / 1e9,
+            "calls": "signrot_calibrate + signrot_build_sign, L2 flushed before each timing"},
+        "gpu_launches": top["gpu_launches"],
+        "clocks": sampler.report(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None) -> int:
     args = parse(argv)
-    return run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_sweep(args) if args.sweep else run_ours(args)
 
 
 if __name__ == "__main__":
