@@ -62,8 +62,8 @@ def test_both_fold_kernels_agree_with_oracle(sr):
     ref = o.calibrate(o.to_f64(x, "bf16"))
     assert ref[0] == k0
     assert run(sr, x_t) == ref  # 16-byte aligned rows, n % 8 == 0: the vector kernel
-    # rows starting 2 bytes past a 16-byte boundary (ld = 4096, n = 4088): the element-wise kernel
-    assert run(sr, x_t[:, 1:4089]) == o.calibrate(o.to_f64(x[:, 1:4089], "bf16"))
+    # rows starting 2 bytes past a 16-byte boundary (ld = 4096, n = 1024): the element-wise kernel
+    assert run(sr, x_t[:, 1:1025]) == o.calibrate(o.to_f64(x[:, 1:1025], "bf16"))
     # n = 28 (n % 8 != 0): the element-wise kernel
     x28 = np.ascontiguousarray(x[:, :28])
     assert run(sr, dev(x28)) == o.calibrate(o.to_f64(x28, "bf16"))
