@@ -50,6 +50,8 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quant", choices=["asym4", "asym8", "sym4", "sym8"], default="asym4",
                     help="grid of the timed kernel: asymmetric INT4 (the metric's), INT8, or symmetric")
+    ap.add_argument("--calib-tokens", type=int, default=None,
+                    help="--sweep: calibration tokens (default 128 x 2048; a multiple of 2048)")
     ap.add_argument("--sweep", action="store_true",
                     help="decode/prefill sweep at n = 14336 (T = 1 .. 32768, latency per call and GB/s, "
                          "warm and after an L2 flush) and the 128 x 2048-token calibration pass; one GPU")
@@ -76,13 +78,17 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "source": "fallback"}
 
 
+# the fused kernels' translation unit and every header it includes
+FUSED_SOURCES = ("rotate_tc.cu", "signrot_device.cuh", "signrot_internal.h", "tc_ptx.cuh")
+
+
 def kernel_sources_digest() -> str:
+    """Digest of the fused kernels' sources: a recorded ncu traffic figure applies while it holds."""
     csrc = os.path.join(ROOT, "rotation_activation_quantization_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + b"\0" + fh.read())
+    for f in FUSED_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -427,7 +433,10 @@ def run_sweep(args) -> int:
 
     x = bf(syn.draw_tokens(w, 0, base)).repeat(Tmax // base, 1)
     d = torch.from_numpy(syn.draw_d(w)).to(dev)
-    xc = bf(syn.draw_calibration(w, 0, base)).repeat(w.calib_T // base, 1)
+    n_cal = args.calib_tokens or w.calib_T
+    if n_cal <= 0 or n_cal % 2048:
+        raise ValueError("--calib-tokens must be a positive multiple of 2048")
+    xc = bf(syn.draw_calibration(w, 0, base)).repeat((n_cal + base - 1) // base, 1)[:n_cal]
     stream = torch.cuda.current_stream(dev)
     ws = torch.empty(n, dtype=torch.int64, device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
@@ -453,14 +462,14 @@ def run_sweep(args) -> int:
         sr.build_sign(n, k, xk, d)
 
     def calib_chunked():
-        for i in range(w.calib_T // 2048):
+        for i in range(n_cal // 2048):
             k, xk, _ = sr.calibrate(xc[i * 2048:(i + 1) * 2048], ws=ws, accumulate=i > 0, t_offset=i * 2048)
         sr.build_sign(n, k, xk, d)
 
     calib_once()
     calib_chunked()
     torch.cuda.synchronize(dev)
-    cal_bytes = w.calib_T * n * 2
+    cal_bytes = n_cal * n * 2
     one_med, one_min = timed(calib_once, 5, True)
     ch_med, _ = timed(calib_chunked, 3, True)
     k, xk, _ = sr.calibrate(xc, ws=ws)
@@ -516,11 +525,11 @@ def run_sweep(args) -> int:
                      "bytes_per_token": bpt, "kernel": "signrot_rotate_quant (T = 32768)",
                      "kernel_sources": kernel_sources_digest()},
         "calibration": {
-            "tokens": w.calib_T, "bytes": cal_bytes,
+            "tokens": n_cal, "bytes": cal_bytes,
             "one_call_ms": one_med, "one_call_gbs": cal_bytes / (one_med * 1e-3) / 1e9,
             "one_call_frac": cal_bytes / (one_med * 1e-3) / 1e9 / peaks["hbm_gbs"],
             "one_call_ms_min": one_min,
-            "chunked_128x2048_ms": ch_med, "chunked_gbs": cal_bytes / (ch_med * 1e-3) / 1e9,
+            "chunked_2048_ms": ch_med, "chunked_gbs": cal_bytes / (ch_med * 1e-3) / 1e9,
             "calls": "signrot_calibrate + signrot_build_sign, L2 flushed before each timing"},
         "gpu_launches": top["gpu_launches"],
         "clocks": sampler.report(),
