@@ -37,7 +37,9 @@ Conventions the pages leave open, and the reading taken here:
   (H_M[b, e] = (-1)^popcount(b & e)); H_28 is Paley's construction I over GF(27) =
   GF(3)[alpha]/(alpha^3 + 2 alpha + 1), field element index e = c0 + 3 c1 + 9 c2, Jacobsthal
   matrix Q[e, f] = chi(e - f), H_28 = I + [[0, 1^T], [-1, Q]] (index 0 is the point at
-  infinity, index 1 + e the field element e).
+  infinity, index 1 + e the field element e). For the explainer's n = 11008 = 344 * 32 no page
+  names the matrix; F = 344 is read as the same construction over GF(343) =
+  GF(7)[alpha]/(alpha^3 + alpha + 1), element index e = c0 + 7 c1 + 49 c2.
 * Column convention y = H x (y_j = sum_i H[j, i] x_i); D acts before H, s after it.
 * s_j = +1 if H[j, k] * D_k * x_k >= 0 else -1, with x_k the signed calibration value of
   channel k at the first token attaining max_t |x_{t,k}|; k is the lowest channel index
@@ -133,7 +135,7 @@ class GF3:
 
 
 GF27 = GF3(3, (1, 2, 0))  # a^3 + 2a + 1
-GF343 = GF3(7, (1, 1, 0))  # a^3 + a + 1 (oracle-only: gives H_344 for the n = 11008 example)
+GF343 = GF3(7, (1, 1, 0))  # a^3 + a + 1: H_344 for the n = 11008 example
 
 
 def paley_skew_hadamard(field: GF3) -> np.ndarray:
@@ -162,8 +164,8 @@ def paley_h28() -> np.ndarray:
 
 @lru_cache(maxsize=None)
 def paley_h344() -> np.ndarray:
-    """Order-344 Paley matrix over GF(343); lets the oracle run the explainer's n = 11008
-    (LLaMA2-7B intermediate size) example as 344 * 32. Not part of the GPU path."""
+    """Order-344 Paley matrix over GF(343) = GF(7)[a]/(a^3 + a + 1), same numbering and border as
+    H_28: the explainer's n = 11008 (LLaMA2-7B intermediate size) token as 344 * 32."""
     h = paley_skew_hadamard(GF343)
     h.setflags(write=False)
     return h
