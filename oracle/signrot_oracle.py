@@ -359,3 +359,43 @@ def rotate_quant(x: np.ndarray, d: np.ndarray, s: np.ndarray | None, bits: int =
     """The whole online path for rows x [T, n] (float64): (packed codes, scale, zero)."""
     codes, scale, zero = quantize_asym(rotate(x, d, s), bits=bits, clip=clip)
     return pack_nibbles(codes), scale, zero
+
+
+# ----------------------------------------------------------------------------------------------
+# consumer side: the down projection that reads the codes. Explainer, "SignRot asks one crowd to
+# walk across the hall": the sign matrix is its own inverse and its flip is folded into the
+# weights offline; "The flip alone does nothing for a symmetric quantizer": the zero-point's
+# correction in the matrix multiply is the zero-point times a precomputed column sum of the
+# weights. The weights' own quantizer (the pages use GPTQ) is out of scope; a per-output-channel
+# symmetric round-to-nearest grid stands in for it.
+# ----------------------------------------------------------------------------------------------
+
+
+def fold_weights(w: np.ndarray, d: np.ndarray, s: np.ndarray | None = None) -> np.ndarray:
+    """W' = W R^T for the down projection out = W x (w is [d_out, n]), R = diag(s) H diag(D) / sqrt(n).
+
+    Then W' (R x) = W R^T R x = W x, R being orthogonal. Row o of W' is R applied to row o of W
+    (W' = W R^T  <=>  W'^T = R W^T), so the fold is the activation rotation of W's rows.
+    """
+    return rotate(w, d, s)
+
+
+def quantize_weights_sym(w: np.ndarray, bits: int = 4):
+    """Per-output-channel symmetric grid for W' rows: (codes int8 [d_out, n], scale f32 [d_out])."""
+    return quantize_sym(w, bits=bits)
+
+
+def w4a4_matmul(codes: np.ndarray, scale: np.ndarray, zero: np.ndarray | None, wcodes: np.ndarray,
+                wscale: np.ndarray) -> np.ndarray:
+    """out[t, o] = scale_t * wscale_o * (sum_j codes[t, j] * wcodes[o, j] - zero_t * c_o),
+    c_o = sum_j wcodes[o, j] (the precomputed column sum); zero = None for a symmetric grid.
+
+    The integer sums are exact in float64 (|sum| < 2^53); the epilogue is float64.
+    """
+    q = np.atleast_2d(np.asarray(codes)).astype(np.float64)
+    wq = np.atleast_2d(np.asarray(wcodes)).astype(np.float64)
+    acc = q @ wq.T
+    if zero is not None:
+        c = wq.sum(axis=1)
+        acc = acc - np.asarray(zero, dtype=np.float64)[:, None] * c[None, :]
+    return acc * np.asarray(scale, dtype=np.float64)[:, None] * np.asarray(wscale, dtype=np.float64)[None, :]
