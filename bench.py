@@ -117,19 +117,25 @@ def cpu_cores() -> int:
     return len(os.sched_getaffinity(0))
 
 
-def oracle_sample(w: syn.Workload, seconds: float, tokens_per_call: int = 8):
-    """Time the CPU oracle (float64 dense rotation + fp32 quantizer) on token blocks until the
-    budget is spent. Returns (tokens/s, tokens, seconds)."""
+def oracle_sample(w: syn.Workload, seconds: float, tokens_per_call: int = 8, fast: bool = False):
+    """Time the CPU oracle (float64 dense rotation + fp32 quantizer; with ``fast`` its O(n log n)
+    cross-check form instead) on token blocks until the budget is spent. The rows are drawn before
+    the clock starts. Returns (tokens/s, tokens, seconds)."""
     from oracle import signrot_oracle as o
 
     d = syn.draw_d(w)
     xc = o.to_f64(syn.draw_calibration(w, 0, min(256, syn.calibration_size(w))), w.dtype)
     k, xk = o.calibrate(xc)
     s = o.build_sign(w.n, k, xk, d)
+    pool = o.to_f64(syn.draw_tokens(w, 0, min(w.T, 256)), w.dtype)
     done, t0 = 0, time.perf_counter()
     while True:
-        x = o.to_f64(syn.draw_tokens(w, done % w.T, done % w.T + tokens_per_call), w.dtype)
-        o.rotate_quant(x, d, s)
+        i = done % (pool.shape[0] - tokens_per_call + 1)
+        x = pool[i:i + tokens_per_call]
+        if fast:
+            o.quantize_asym(o.rotate_fast(x, d, s))
+        else:
+            o.rotate_quant(x, d, s)
         done += x.shape[0]
         el = time.perf_counter() - t0
         if el >= seconds:
@@ -192,35 +198,40 @@ class ClockSampler:
 
 
 def run_reference(args) -> int:
+    """The reference arm: the float64 oracle on the host cores, exactly K timed steps after W
+    untimed ones, each step a sample of the workload's rows sized so the run stays within a few
+    minutes (1 to 4 tokens per step)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     w = workload(args)
     cores = cpu_cores()
-    tokens_per_step = 4
     from oracle import signrot_oracle as o
 
     d = syn.draw_d(w)
     xc = o.to_f64(syn.draw_calibration(w, 0, min(256, syn.calibration_size(w))), w.dtype)
     k, xk = o.calibrate(xc)
     s = o.build_sign(w.n, k, xk, d)
-    xs = o.to_f64(syn.draw_tokens(w, 0, tokens_per_step), w.dtype)
+    xs = o.to_f64(syn.draw_tokens(w, 0, 4), w.dtype)
+    o.rotate_quant(xs[:1], d, s)  # builds and caches the dense H
     t0 = time.perf_counter()
-    for _ in range(max(args.warmup, 1) if args.warmup else 0):
-        o.rotate_quant(xs, d, s)
-    step_s = max((time.perf_counter() - t0) / max(args.warmup, 1), 1e-6)
+    o.rotate_quant(xs[:1], d, s)
+    per_token = max(time.perf_counter() - t0, 1e-6)
     budget = 150.0
-    steps = max(1, min(args.steps, int(budget / step_s)))
+    K, W = max(args.steps, 1), max(args.warmup, 0)
+    tokens_per_step = int(max(1, min(4, budget / ((K + W) * per_token))))
+    xs = xs[:tokens_per_step]
+    for _ in range(W):
+        o.rotate_quant(xs, d, s)
     t0 = time.perf_counter()
-    for _ in range(steps):
+    for _ in range(K):
         o.rotate_quant(xs, d, s)
     el = time.perf_counter() - t0
-    value = tokens_per_step * steps / el
+    value = tokens_per_step * K / el
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": steps, "steps_requested": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * el / steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "steps": K, "warmup": W, "ms_per_step": 1e3 * el / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "n": w.n, "tokens_per_step": tokens_per_step,
                    "input_dtype": w.dtype},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -399,6 +410,10 @@ def run_ours(args) -> int:
             line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                                     "sample": f"{done} tokens of {w.name} in {el:.1f} s (float64 dense "
                                               f"O(n^2) rotation + fp32 quantizer)"}
+            vf, donef, elf = oracle_sample(w, min(3.0, args.cpu_seconds), fast=True)
+            line["cpu_fast_form"] = {"value": vf, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                                     "sample": f"{donef} tokens of {w.name} in {elf:.1f} s (the oracle's "
+                                               f"O(n log n) cross-check form: H_F block + FWHT, float64)"}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

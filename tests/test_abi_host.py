@@ -127,3 +127,21 @@ def test_error_messages(binding):
     assert b"n = 1000" in lib.signrot_last_error()
     for st in range(6):
         assert lib.signrot_status_string(st)
+
+
+def test_bench_reference_arm_prints_the_contract_line():
+    """bench.py --impl reference on the CPU: one JSON line with the contract's keys, K steps."""
+    import json
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--config", "2",
+                          "--steps", "3", "--warmup", "1"], capture_output=True, text=True, check=True,
+                         cwd=root, timeout=600).stdout.strip().splitlines()
+    line = json.loads(out[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e", "impl"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["steps"] == 3 and line["warmup"] == 1
+    assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["workload"]
