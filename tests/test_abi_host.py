@@ -145,3 +145,23 @@ def test_bench_reference_arm_prints_the_contract_line():
     assert line["impl"] == "reference" and line["steps"] == 3 and line["warmup"] == 1
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["workload"]
+
+
+def test_bench_bytes_per_token():
+    """Algorithmic bytes per token: bf16 row in, codes out, fp32 scale (+ zero). C3 and C4 give the
+    35 848 and 71 688 B of the measurement plan; INT8 and symmetric grids move accordingly."""
+    import importlib.util
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(root, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    from rotation_activation_quantization_b200 import synthetic as syn
+
+    w3, w4, w1 = syn.workload(3), syn.workload(4), syn.workload(1)
+    assert bench.bytes_per_token(w3) == 35848
+    assert bench.bytes_per_token(w4) == 71688
+    assert bench.bytes_per_token(w1) == 4 * 1024 + 512 + 8  # fp32 rows
+    assert bench.bytes_per_token(w3, "asym8") == 2 * 14336 + 14336 + 8
+    assert bench.bytes_per_token(w3, "sym4") == 2 * 14336 + 7168 + 4
+    assert bench.bytes_per_token(w3, "sym8") == 2 * 14336 + 14336 + 4
