@@ -10,7 +10,8 @@ once before timing; its time is reported separately under "calibration". Multi-G
 tokens (weak scaling: every rank processes its own T tokens, no data-path collective).
 
 Rank 0 prints one JSON line. --impl reference times the float64 CPU oracle on a bounded sample
-of the same workload (the baseline this build is measured against).
+of the same workload (a reported CPU baseline). --quant picks another grid of the same kernels;
+--sweep measures the decode/prefill T sweep and the long calibration pass at n = 14336.
 """
 from __future__ import annotations
 

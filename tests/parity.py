@@ -140,7 +140,7 @@ def check_quant(q_gpu: np.ndarray, scale_gpu: np.ndarray, zero_gpu: np.ndarray |
     tie = _half_dist(vpre.astype(np.float64)) < window
     allowed_step = 1 + np.floor(window)
     hard = mism & ~((np.abs(diff) <= allowed_step) & tie)
-    wide = window > 0.5  # rounding noise spans whole codes: judge by the dequantized value
+    wide = window > 0.5  # rounding noise spans whole codes: decide by the dequantized value
     if wide.any():
         hard = hard & ~wide
     assert not hard.any(), (f"{int(hard.sum())} code mismatches away from ties, first at "
