@@ -44,7 +44,8 @@ def parse(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=3, help="workload index (1..5); 3 = LLaMA3-8B down_proj")
+    ap.add_argument("--config", type=int, default=3,
+                    help="workload index (1..6); 3 = LLaMA3-8B down_proj, 6 = LLaMA2-7B (n = 11008)")
     ap.add_argument("--tokens", type=int, default=None, help="override tokens per GPU")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle sample budget")

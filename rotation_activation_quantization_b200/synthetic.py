@@ -76,6 +76,11 @@ WORKLOADS = {
     5: _wl(5, name="llama3_8b_down_proj_n14336_sweep_bf16", n=14336, T=32768, dtype="bf16",
            base="laplace", sigma=0.2, outlier_lo=800.0, outlier_hi=2000.0, outlier_frac=0.95,
            secondaries=8, sec_lo=20.0, sec_hi=60.0, calib_T=128 * 2048),
+    # LLaMA-2-7B's down projection (n = 11008 = 344 * 32, H_344 kron H_32): the explainer's token
+    # of paragraph "Here is how it breaks" (outlier 1510) sits inside the outlier range
+    6: _wl(6, name="llama2_7b_down_proj_n11008_T8192_bf16", n=11008, T=8192, dtype="bf16",
+           base="laplace", sigma=0.2, outlier_lo=1000.0, outlier_hi=2000.0, outlier_frac=0.95,
+           secondaries=8, sec_lo=20.0, sec_hi=60.0, calib_T=2048),
 }
 
 SWEEP_T = (1, 8, 64, 256, 1024, 4096, 32768)

@@ -234,7 +234,7 @@ def test_calibrate_brute_force_random_tiny():
         assert o.calibrate(x) == (best[1], best[2])
 
 
-@pytest.mark.parametrize("index", [1, 2, 3, 4])
+@pytest.mark.parametrize("index", [1, 2, 3, 4, 6])
 def test_calibration_finds_planted_channel(index):
     w = syn.workload(index)
     xc = o.to_f64(syn.draw_calibration(w, 0, min(256, syn.calibration_size(w))), w.dtype)
