@@ -50,8 +50,9 @@ Conventions the pages leave open, and the reading taken here:
   scales lo and hi (c = 1 is the only ratio the workloads use).
 * Codes are unsigned 0..15; element 2i goes to the low nibble of byte i, 2i+1 to the high one.
 
-Every function here is pinned by the CPU tests (tests/test_oracle_pins.py) against closed forms,
-invariants, brute force on tiny inputs, or numbers printed on the pages.
+Every function here is pinned by the CPU tests (tests/test_oracle_pins.py; the consumer side in
+tests/test_oracle_consumer.py) against closed forms, invariants, brute force on tiny inputs, or
+numbers printed on the pages.
 """
 from __future__ import annotations
 
