@@ -92,9 +92,13 @@ signrot_status signrot_calibrate(const void* x, int32_t dtype, int64_t T, int32_
  * takes the same arguments as signrot_calibrate minus ws, and keeps the per-channel keys in a
  * fixed array inside the library's device image (SIGNROT_STATIC_SCRATCH_MAX_N channels, 256 KB,
  * held on every GPU that loads the library until the process exits). It allocates nothing.
- *   - n > SIGNROT_STATIC_SCRATCH_MAX_N returns SIGNROT_ERR_UNSUPPORTED with a message.
+ *   - Arguments are checked as for signrot_calibrate, before any CUDA call. The array holds
+ *     every supported row length; an n beyond SIGNROT_STATIC_SCRATCH_MAX_N is not a supported
+ *     form and returns SIGNROT_ERR_UNSUPPORTED_N with a message.
  *   - The first call on a device looks the array's device address up (cudaGetSymbolAddress with
- *     that device current) and caches it; make that first call before any stream capture.
+ *     that device current) and caches it; make that first call before any stream capture. The
+ *     cache assumes the device's primary context is never reset: after cudaDeviceReset the
+ *     library image is reloaded and this entry point must not be called again in that process.
  *   - All calls on a device share the one array, and it keeps the last call's contents:
  *     accumulate == 0 clears it first; accumulate != 0 folds into whatever the previous call on
  *     that device left there. Calls that overlap on the GPU (other streams, other host threads)

@@ -12,7 +12,9 @@
 // is part of the module's device image: every GPU that loads the library holds it until the
 // process exits. Host code cannot use the array's name as a device address, so the first call on
 // each device looks the address up with cudaGetSymbolAddress (with that device current) and
-// caches it; later calls reuse the cached address.
+// caches it; later calls reuse the cached address. The cache is keyed by device ordinal and
+// assumes the device's primary context lives as long as the process: after a cudaDeviceReset the
+// module is loaded again, possibly at another address, and the cached one must not be used.
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
@@ -64,6 +66,12 @@ signrot_status scratch_address(uint64_t** out) {
 extern "C" signrot_status signrot_calibrate_static(const void* x, int32_t dtype, int64_t T, int32_t n,
                                                    int64_t ld, int64_t t_offset, int32_t accumulate,
                                                    int32_t* k_out, float* xk_out, void* stream) {
+  // every argument is checked before any CUDA call, as for the workspace-taking entry point
+  signrot_status st = signrot::check_calibrate_args(x, dtype, T, n, ld, t_offset, k_out, xk_out);
+  if (st != SIGNROT_OK) return st;
+  // The array covers every supported row length (the longest is 2^15), so this guard only fires
+  // if the two ever drift apart; an unsupported n has already been refused above.
+  static_assert(SIGNROT_STATIC_SCRATCH_MAX_N >= (1 << 15), "the static array must hold the longest row");
   if (n > SIGNROT_STATIC_SCRATCH_MAX_N) {
     char msg[160];
     std::snprintf(msg, sizeof(msg),
@@ -71,10 +79,10 @@ extern "C" signrot_status signrot_calibrate_static(const void* x, int32_t dtype,
                   "use signrot_calibrate with a caller workspace",
                   n, SIGNROT_STATIC_SCRATCH_MAX_N);
     signrot::set_last_error(msg);
-    return SIGNROT_ERR_UNSUPPORTED;
+    return SIGNROT_ERR_UNSUPPORTED_N;
   }
   uint64_t* ws = nullptr;
-  const signrot_status st = scratch_address(&ws);
+  st = scratch_address(&ws);
   if (st != SIGNROT_OK) return st;
   return signrot_calibrate(x, dtype, T, n, ld, t_offset, ws, accumulate, k_out, xk_out, stream);
 }

@@ -219,16 +219,10 @@ extern "C" {
 signrot_status signrot_calibrate(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
                                  int64_t t_offset, uint64_t* ws, int32_t accumulate,
                                  int32_t* k_out, float* xk_out, void* stream) {
-  g_last_error[0] = '\0';
-  signrot::Shape sh;
-  signrot_status st = check_rows(x, dtype, T, n, ld, &sh);
+  signrot_status st = signrot::check_calibrate_args(x, dtype, T, n, ld, t_offset, k_out, xk_out);
   if (st != SIGNROT_OK) return st;
-  if (ws == nullptr || k_out == nullptr || xk_out == nullptr)
-    return fail(SIGNROT_ERR_INVALID_ARG, "ws, k_out and xk_out must be device pointers");
-  if (!aligned(ws, 8) || !aligned(k_out, 4) || !aligned(xk_out, 4))
-    return fail(SIGNROT_ERR_ALIGNMENT, "ws (8 B), k_out and xk_out (4 B) misaligned");
-  if (t_offset < 0 || t_offset + T > 0x7fffffffLL)
-    return fail(SIGNROT_ERR_INVALID_ARG, "token indices t_offset + t must stay below 2^31 - 1");
+  if (ws == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "ws must be a device pointer");
+  if (!aligned(ws, 8)) return fail(SIGNROT_ERR_ALIGNMENT, "ws is not 8-byte aligned");
   auto s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (!accumulate) {
@@ -434,6 +428,15 @@ void signrot::set_last_error(const char* msg) {
   std::snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
 }
 
-extern "C" {
-
-}  // extern "C"
+signrot_status signrot::check_calibrate_args(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld,
+                                             int64_t t_offset, const int32_t* k_out, const float* xk_out) {
+  g_last_error[0] = '\0';
+  signrot::Shape sh;
+  signrot_status st = check_rows(x, dtype, T, n, ld, &sh);
+  if (st != SIGNROT_OK) return st;
+  if (k_out == nullptr || xk_out == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "k_out and xk_out must be device pointers");
+  if (!aligned(k_out, 4) || !aligned(xk_out, 4)) return fail(SIGNROT_ERR_ALIGNMENT, "k_out and xk_out must be 4-byte aligned");
+  if (t_offset < 0 || t_offset + T > 0x7fffffffLL)
+    return fail(SIGNROT_ERR_INVALID_ARG, "token indices t_offset + t must stay below 2^31 - 1");
+  return SIGNROT_OK;
+}

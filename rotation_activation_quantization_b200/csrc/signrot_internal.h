@@ -13,6 +13,11 @@ void count_launch(int n = 1);
 // Sets the message signrot_last_error returns on this host thread.
 void set_last_error(const char* msg);
 
+// The argument checks signrot_calibrate makes on everything but its workspace (rows, n, outputs,
+// token offsets); clears the last-error message first, sets it on failure. No CUDA call.
+int32_t check_calibrate_args(const void* x, int32_t dtype, int64_t T, int32_t n, int64_t ld, int64_t t_offset,
+                             const int32_t* k_out, const float* xk_out);
+
 // Library-owned Paley matrices (paley.cpp), row-major, entries +/-1.
 void paley_h28(int8_t h[28][28]);
 void paley_h344(int8_t* h);  // [344 * 344]

@@ -14,7 +14,7 @@ import pytest
 from oracle import signrot_oracle as o
 from rotation_activation_quantization_b200 import synthetic as syn
 
-from parity import check_quant, check_rotation, record
+from parity import check_quant, check_rotation, oracle_sign, record
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -63,7 +63,7 @@ def test_f344_parity(sr, n, dtype):
     q, scale, zero = sr.rotate_quant(x_t, d_t, s_t)
     q2, scale2, zero2 = sr.rotate_quant_outlier(x_t, d_t, k, xk)
     assert torch.equal(q, q2) and torch.equal(scale, scale2) and torch.equal(zero, zero2)
-    st.update(check_quant(q.cpu().numpy(), scale.cpu().numpy(), zero.cpu().numpy(), y_ref, x64=x64, strict=False))
+    st.update(check_quant(q.cpu().numpy(), scale.cpu().numpy(), zero.cpu().numpy(), y_ref, x64=x64))
     for bits, sym in [(8, False), (4, True), (8, True)]:
         if sym:
             qv, sv = sr.rotate_quant_sym_outlier(x_t, d_t, k, xk, bits=bits)
@@ -72,7 +72,7 @@ def test_f344_parity(sr, n, dtype):
             qv, sv, zv = sr.rotate_quant_outlier(x_t, d_t, k, xk, bits=bits)
         torch.cuda.synchronize()
         check_quant(qv.cpu().numpy(), sv.cpu().numpy(), None if zv is None else zv.cpu().numpy(), y_ref,
-                    x64=x64, strict=False, bits=bits, sym=sym)
+                    x64=x64, bits=bits, sym=sym)
     record(f"f344_{dtype}_{n}", {**st, "plain_rel_l2_max": st_plain["rel_l2_max"]})
 
 
@@ -104,10 +104,12 @@ def test_f344_ragged_and_host_buffers(sr):
         k, xk, _ = sr.calibrate(x_t)
         s_t = sr.build_sign(n, k, xk, d_t)
         x64 = o.to_f64(x, "bf16")
-        y_ref = o.rotate(x64, d, s_t.cpu().numpy())
+        s_ref = oracle_sign(x64, d)
+        assert (s_t.cpu().numpy() == s_ref).all()
+        y_ref = o.rotate(x64, d, s_ref)
         q, scale, zero = sr.rotate_quant(x_t, d_t, s_t)
         torch.cuda.synchronize()
-        check_quant(q.cpu().numpy(), scale.cpu().numpy(), zero.cpu().numpy(), y_ref, x64=x64, strict=False)
+        check_quant(q.cpu().numpy(), scale.cpu().numpy(), zero.cpu().numpy(), y_ref, x64=x64)
         xh = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
         qh = torch.empty((T, n // 2), dtype=torch.uint8).pin_memory()
         sh = torch.empty(T, dtype=torch.float32).pin_memory()

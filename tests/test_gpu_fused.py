@@ -7,7 +7,7 @@ import pytest
 from oracle import signrot_oracle as o
 from rotation_activation_quantization_b200 import synthetic as syn
 
-from parity import check_quant, check_rotation, record
+from parity import check_quant, check_rotation, oracle_sign, record
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -49,9 +49,11 @@ def test_outlier_entry_equals_sign_vector_entry(sr, n):
     y2 = sr.rotate_outlier(x_t, d_t, k, xk)
     assert torch.equal(y1, y2)
     x64 = o.to_f64(x, "bf16")
-    y_ref = o.rotate(x64, d, s_t.cpu().numpy())
+    s_ref = oracle_sign(x64, d)
+    assert (s_t.cpu().numpy() == s_ref).all()
+    y_ref = o.rotate(x64, d, s_ref)
     st = check_rotation(y2.cpu().numpy(), y_ref)
-    st.update(check_quant(q2.cpu().numpy(), s2.cpu().numpy(), z2.cpu().numpy(), y_ref, x64=x64, strict=False))
+    st.update(check_quant(q2.cpu().numpy(), s2.cpu().numpy(), z2.cpu().numpy(), y_ref, x64=x64))
     record(f"fused_outlier_{n}", st)
     assert sr.device_error() == 0
 
@@ -65,11 +67,11 @@ def test_token_counts_around_the_grid(sr, T):
     q, scale, zero = sr.rotate_quant_outlier(x_t, d_t, k, xk)
     torch.cuda.synchronize()
     rows = sorted({0, T // 2, T - 1})
+    s = oracle_sign(o.to_f64(x, "bf16"), d)
     x64 = o.to_f64(x[rows], "bf16")
-    s = o.build_sign(n, int(k.item()), float(xk.item()), d)
     y_ref = o.rotate(x64, d, s)
     qn, sn, zn = q.cpu().numpy(), scale.cpu().numpy(), zero.cpu().numpy()
-    record(f"fused_T{T}", check_quant(qn[rows], sn[rows], zn[rows], y_ref, x64=x64, strict=False))
+    record(f"fused_T{T}", check_quant(qn[rows], sn[rows], zn[rows], y_ref, x64=x64))
     assert sr.device_error() == 0
 
 
@@ -83,11 +85,11 @@ def test_general_sign_vector_on_fused_path(sr, n):
     y_ref = o.rotate(x64, d, s)
     check_rotation(sr.rotate(x_t, d_t, s_t).cpu().numpy(), y_ref)
     q, scale, zero = sr.rotate_quant(x_t, d_t, s_t)
-    check_quant(q.cpu().numpy(), scale.cpu().numpy(), zero.cpu().numpy(), y_ref, x64=x64, strict=False)
+    check_quant(q.cpu().numpy(), scale.cpu().numpy(), zero.cpu().numpy(), y_ref, x64=x64)
     # and with no sign adjustment at all
     y_ref0 = o.rotate(x64, d)
     q, scale, zero = sr.rotate_quant(x_t, d_t, None)
-    check_quant(q.cpu().numpy(), scale.cpu().numpy(), zero.cpu().numpy(), y_ref0, x64=x64, strict=False)
+    check_quant(q.cpu().numpy(), scale.cpu().numpy(), zero.cpu().numpy(), y_ref0, x64=x64)
     assert sr.device_error() == 0
 
 

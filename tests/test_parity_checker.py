@@ -62,3 +62,49 @@ def test_wrong_symmetric_scale_fails():
     bad[2] *= 1.0001
     with pytest.raises(AssertionError):
         check_quant(encode(codes, 4, True), bad, None, y, bits=4, sym=True)
+
+
+def _outlier_rows(n=4096, T=64):
+    from rotation_activation_quantization_b200 import synthetic as syn
+
+    x, d, _ = syn.random_rows(n, T, "bf16", seed=17, outlier=1500.0)
+    x64 = o.to_f64(x, "bf16")
+    k, xk = o.calibrate(x64)
+    y = o.rotate_fast(x64, d, o.build_sign(n, k, xk, d))
+    return x64, y
+
+
+def _flip_ties(codes, vpre, count):
+    """Move `count` codes that sit at a rounding tie to the other neighbour of the tie."""
+    c = codes.astype(np.int32).copy()
+    frac = vpre - np.floor(vpre)
+    ties = np.argwhere((np.abs(frac - 0.5) < 1e-3) & (c > 0) & (c < 15))
+    assert len(ties) >= count
+    for t, j in ties[:count]:
+        fl = int(np.floor(vpre[t, j]))
+        c[t, j] = fl + 1 if c[t, j] == fl else fl
+    return c
+
+
+def test_tie_cap_holds_on_rows_with_a_massive_outlier():
+    """Rows whose rotation carries a massive outlier's shift are held to the 1e-4 tie cap, with the
+    input rows given: a few tie flips pass, one more than the cap fails."""
+    x64, y = _outlier_rows()
+    codes, scale, zero = o.quantize_asym(y)
+    vpre, _ = o.asym_preround(y)
+    cap = int(np.ceil(1e-4 * y.size))
+    ok = _flip_ties(codes, vpre, cap)
+    st = check_quant(encode(ok, 4, False), scale, zero, y, x64=x64)
+    assert st["ill_conditioned_tokens"] == 0 and st["well_mismatches"] == cap
+    bad = _flip_ties(codes, vpre, cap + 1)
+    with pytest.raises(AssertionError):
+        check_quant(encode(bad, 4, False), scale, zero, y, x64=x64)
+
+
+def test_scale_bar_is_not_widened_on_long_outlier_rows():
+    x64, y = _outlier_rows()
+    codes, scale, zero = o.quantize_asym(y)
+    bad = scale.copy()
+    bad[5] *= 1 + 3e-5
+    with pytest.raises(AssertionError):
+        check_quant(encode(codes, 4, False), bad, zero, y, x64=x64)

@@ -74,10 +74,38 @@ def test_two_consecutive_fresh_calls_clear_the_shared_array(lib):
     assert _call_static(lib, small, 0, 0) == _call_workspace(lib, small, ws_small, 0, 0)
 
 
-def test_rejects_rows_longer_than_the_static_array(lib):
+def test_longest_row_and_no_device_allocation(lib):
+    """The longest supported row (n = 32768, the array's full size) equals the workspace entry
+    point, and a warmed-up call leaves the device's free memory unchanged: it allocates nothing."""
+    n = 32768
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn((300, n), generator=g) * 0.3).to(torch.bfloat16)
+    x[123, 31000] = 2500.0
+    x = x.cuda()
+    ws = torch.empty(n, dtype=torch.int64, device="cuda")
+    expect = _call_workspace(lib, x, ws, 0, 0)
+    assert expect[0] == 31000
+    assert _call_static(lib, x, 0, 0) == expect
+    k = torch.empty(1, dtype=torch.int32, device="cuda")
+    xk = torch.empty(1, dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        st = lib.signrot_calibrate_static(x.data_ptr(), 0, 300, n, n, 0, 0, k.data_ptr(), xk.data_ptr(),
+                                          torch.cuda.current_stream().cuda_stream)
+        assert st == 0, lib.signrot_last_error()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert int(k.item()) == 31000
+
+
+def test_rejects_unsupported_rows_before_touching_the_device(lib):
     x = torch.zeros((2, 65536), dtype=torch.bfloat16, device="cuda")
     k = torch.empty(1, dtype=torch.int32, device="cuda")
     xk = torch.empty(1, dtype=torch.float32, device="cuda")
     st = lib.signrot_calibrate_static(x.data_ptr(), 0, 2, 65536, 65536, 0, 0, k.data_ptr(), xk.data_ptr(), None)
-    assert st == 5
-    assert b"static workspace" in lib.signrot_last_error()
+    assert st == 2  # the same status signrot_calibrate gives for this n
+    assert b"65536" in lib.signrot_last_error()
+    st = lib.signrot_calibrate_static(None, 0, 2, 4096, 4096, 0, 0, k.data_ptr(), xk.data_ptr(), None)
+    assert st == 1
