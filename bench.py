@@ -1,13 +1,16 @@
 #!/usr/bin/env python
 """Throughput of the fused SignRot online path (rotate + sign-adjust + asymmetric INT4 quant).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 3]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 4] [--also 3]
 
 One step = one pass of the online path over the workload's T tokens resident in HBM
-(signrot_rotate_quant on [T, n] bf16 rows -> packed INT4 codes + fp32 scale/zero). The outlier
-channel and sign vector come from a calibration pass (signrot_calibrate + signrot_build_sign) run
-once before timing; its time is reported separately under "calibration". Multi-GPU runs shard
-tokens (weak scaling: every rank processes its own T tokens, no data-path collective).
+(signrot_rotate_quant on [T, n] bf16 rows -> packed INT4 codes + fp32 scale/zero). The default
+workload is LLaMA-3-70B's down projection (n = 28672, T = 16384 per GPU), the largest one that
+fits one GPU; LLaMA-3-8B's (n = 14336, T = 8192) is measured the same way and reported under
+"also". The outlier channel and sign vector come from a calibration pass (signrot_calibrate +
+signrot_build_sign) run once before timing; its time is reported separately under
+"calibration". Multi-GPU runs shard tokens (weak scaling: every rank processes its own T tokens,
+no data-path collective).
 
 Rank 0 prints one JSON line. --impl reference times the float64 CPU oracle on a bounded sample
 of the same workload (a reported CPU baseline). --quant picks another grid of the same kernels;
@@ -36,6 +39,7 @@ from rotation_activation_quantization_b200 import synthetic as syn  # noqa: E402
 METRIC = "tokens/s and achieved HBM GB/s (% of B200 peak) for fused rotate+INT4 quant"
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal
 
 
 def parse(argv=None):
@@ -44,8 +48,12 @@ def parse(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=3,
-                    help="workload index (1..6); 3 = LLaMA3-8B down_proj, 6 = LLaMA2-7B (n = 11008)")
+    ap.add_argument("--config", type=int, default=4,
+                    help="workload index (1..6); 4 = LLaMA3-70B down_proj (n = 28672, the largest single-GPU "
+                         "workload), 3 = LLaMA3-8B (n = 14336), 6 = LLaMA2-7B (n = 11008)")
+    ap.add_argument("--also", type=lambda v: [int(i) for i in v.split(",") if i], default=None,
+                    help="comma-separated workloads measured the same way and reported under 'also' "
+                         "(default: 3 beside the default workload, none otherwise)")
     ap.add_argument("--tokens", type=int, default=None, help="override tokens per GPU")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle sample budget")
@@ -58,6 +66,11 @@ def parse(argv=None):
                     help="decode/prefill sweep at n = 14336 (T = 1 .. 32768, latency per call and GB/s, "
                          "warm and after an L2 flush) and the 128 x 2048-token calibration pass; one GPU")
     return ap.parse_args(argv)
+
+
+def _default_also(args) -> None:
+    if args.also is None:
+        args.also = [3] if (args.config == 4 and not args.tokens) else []
 
 
 def workload(args) -> syn.Workload:
@@ -177,7 +190,7 @@ class ClockSampler:
             except Exception as e:
                 self.err = f"{type(e).__name__}: {e}"
                 return
-            time.sleep(0.002)
+            time.sleep(0.0005)
 
     def __enter__(self):
         if self.h is not None:
@@ -245,6 +258,129 @@ def run_reference(args) -> int:
     return 0
 
 
+def _to_dev(torch, a: np.ndarray, dtype: str, dev):
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def measure_kernel(torch, sr, w: syn.Workload, args, dev, world: int, rank: int, quant: str) -> dict:
+    """Device time of K launches of the fused call over this rank's T tokens of workload w.
+
+    Inputs larger than L2: K back-to-back launches between one event pair (an event recorded
+    between two launches would also stop the next launch from being scheduled while the previous
+    one drains). Inputs that fit in L2: each launch timed alone by its own event pair after a
+    write larger than L2 (flushed), and the K launches back to back as well (warm, reported
+    beside it)."""
+    import torch.distributed as dist
+
+    T, n = w.T, w.n
+    x_np = syn.draw_tokens(w, *sharding.weak_shard(rank, T))
+    d_np = syn.draw_d(w)
+    xc_np = syn.draw_calibration(w)
+    x = _to_dev(torch, x_np, w.dtype, dev)
+    d = torch.from_numpy(d_np).to(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # calibration (once per model; timed on its own)
+    xc = _to_dev(torch, xc_np, w.dtype, dev)
+    ws = torch.empty(n, dtype=torch.int64, device=dev)
+    for _ in range(2):
+        k, xk, _ = sr.calibrate(xc, ws=ws)
+        s = sr.build_sign(n, k, xk, d)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    k, xk, _ = sr.calibrate(xc, ws=ws)
+    s = sr.build_sign(n, k, xk, d)
+    c1.record(stream)
+    torch.cuda.synchronize(dev)
+    calib_ms = c0.elapsed_time(c1)
+    del xc, s
+
+    bits = 8 if quant.endswith("8") else 4
+    sym = quant.startswith("sym")
+    q = torch.empty((T, n * bits // 8), dtype=torch.int8 if (sym and bits == 8) else torch.uint8, device=dev)
+    scale = torch.empty(T, dtype=torch.float32, device=dev)
+    zero = torch.empty(T, dtype=torch.float32, device=dev)
+
+    def step():
+        if sym:
+            sr.rotate_quant_sym_outlier(x, d, k, xk, bits=bits, q=q, scale=scale)
+        else:
+            sr.rotate_quant_outlier(x, d, k, xk, bits=bits, q=q, scale=scale, zero=zero)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    bpt = bytes_per_token(w, quant)
+    resident = T * bpt < 2 * L2_BYTES
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if resident else None
+    sampler = ClockSampler(dev.index)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = sr.kernel_launches()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        if resident:
+            ms = 0.0
+            for _ in range(K):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                step()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                ms += e0.elapsed_time(e1)
+            region_ms = ms
+        else:
+            ev0.record(stream)
+            for _ in range(K):
+                step()
+            ev1.record(stream)
+            torch.cuda.synchronize(dev)
+            region_ms = ev0.elapsed_time(ev1)
+    launches = sr.kernel_launches() - launches0
+    warm_ms = None
+    if resident:  # the same launches back to back with the inputs left in L2
+        ev0.record(stream)
+        for _ in range(K):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        warm_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        dist.barrier()
+    region_ms_max = sharding.max_over_ranks(region_ms, device=dev)
+    avg_launch_ms = region_ms / K  # the fused kernel is the only launch in the region
+    achieved = bpt * T / (avg_launch_ms * 1e-3) / 1e9
+    return {"w": w, "x_np": x_np, "x": x, "d": d, "k": k, "xk": xk, "region_ms": region_ms,
+            "region_ms_max": region_ms_max, "avg_launch_ms": avg_launch_ms, "achieved": achieved, "bpt": bpt,
+            "launches": launches, "calib_ms": calib_ms, "calib_tokens": int(xc_np.shape[0]), "sampler": sampler,
+            "resident": resident, "warm_ms": warm_ms, "sym": sym}
+
+
+def roofline_entry(m: dict, quant: str, peaks: dict, digest: str) -> dict:
+    w = m["w"]
+    traffic = recorded_traffic(w, digest) if quant == "asym4" else None
+    return {"bound": "hbm", "achieved": m["achieved"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": m["achieved"] / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peaks["source"],
+            "frac_of_nominal_8tbs": m["achieved"] / NOMINAL_HBM_GBS,
+            "bytes_per_token": m["bpt"], "tokens_per_launch": w.T,
+            "kernel": "signrot_rotate_quant" if not m["sym"] else "signrot_rotate_quant_sym",
+            "kernel_sources": digest, "launch_ms_mean": m["avg_launch_ms"]}
+
+
+def l2_note(m: dict) -> str:
+    mb = m["bpt"] * m["w"].T / 1e6
+    if m["resident"]:
+        return (f"inputs fit in L2 ({mb:.1f} MB per step vs {L2_BYTES / 1e6:.0f} MB): each launch timed "
+                f"alone after a {2 * L2_BYTES / 1e6:.0f} MB L2-flushing write; warm back-to-back rate beside it")
+    return f"inputs larger than L2 ({mb:.1f} MB per step vs {L2_BYTES / 1e6:.0f} MB), no flush"
+
+
 def run_ours(args) -> int:
     import torch
     import torch.distributed as dist
@@ -264,78 +400,18 @@ def run_ours(args) -> int:
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
         dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
     sr.lib()
+    stream = torch.cuda.current_stream(dev)
 
     w = workload(args)
     T, n = w.T, w.n
-    # inputs: this rank's own T tokens (weak scaling), D, and the calibration batch
-    x_np = syn.draw_tokens(w, *sharding.weak_shard(rank, T))
-    d_np = syn.draw_d(w)
-    xc_np = syn.draw_calibration(w)
-
-    def to_dev(a):
-        if w.dtype == "bf16":
-            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
-        return torch.from_numpy(a).to(dev)
-
-    x = to_dev(x_np)
-    d = torch.from_numpy(d_np).to(dev)
-    stream = torch.cuda.current_stream(dev)
-
-    # calibration (once per model; timed on its own)
-    xc = to_dev(xc_np)
-    ws = torch.empty(n, dtype=torch.int64, device=dev)
-    for _ in range(2):
-        k, xk, _ = sr.calibrate(xc, ws=ws)
-        s = sr.build_sign(n, k, xk, d)
-    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    c0.record(stream)
-    k, xk, _ = sr.calibrate(xc, ws=ws)
-    s = sr.build_sign(n, k, xk, d)
-    c1.record(stream)
-    torch.cuda.synchronize(dev)
-    calib_ms = c0.elapsed_time(c1)
-    del xc
-
-    bits = 8 if args.quant.endswith("8") else 4
-    sym = args.quant.startswith("sym")
-    q = torch.empty((T, n * bits // 8), dtype=torch.int8 if (sym and bits == 8) else torch.uint8, device=dev)
-    scale = torch.empty(T, dtype=torch.float32, device=dev)
-    zero = torch.empty(T, dtype=torch.float32, device=dev)
-
-    def step():
-        if sym:
-            sr.rotate_quant_sym_outlier(x, d, k, xk, bits=bits, q=q, scale=scale)
-        else:
-            sr.rotate_quant_outlier(x, d, k, xk, bits=bits, q=q, scale=scale, zero=zero)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-
-    K = args.steps
-    # one event pair around the K back-to-back launches: an event recorded between two launches
-    # would also stop the next launch from being scheduled while the previous one drains
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    launches0 = sr.kernel_launches()
-    with sampler:
-        ev0.record(stream)
-        for i in range(K):
-            step()
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
-    launches = sr.kernel_launches() - launches0
-    if world > 1:
-        dist.barrier()
-    region_ms = ev0.elapsed_time(ev1)
-    region_ms_max = sharding.max_over_ranks(region_ms, device=dev)
+    m = measure_kernel(torch, sr, w, args, dev, world, rank, args.quant)
+    x_np, d, k, xk = m["x_np"], m["d"], m["k"], m["xk"]
+    h2d = m["x"].numel() * m["x"].element_size()
+    del m["x"]
 
     # end to end through the host-buffer C-ABI call: pinned host rows -> HBM -> fused kernel ->
     # pinned host codes, chunked over two streams so copies overlap (the copies are timed)
-    E = args.e2e_steps or max(3, min(K, 20))
+    E = args.e2e_steps or max(3, min(args.steps, 20))
     xh = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16) if w.dtype == "bf16" else torch.from_numpy(x_np)
     xh = xh.pin_memory()
     qh = torch.empty((T, n // 2), dtype=torch.uint8).pin_memory()
@@ -361,21 +437,26 @@ def run_ours(args) -> int:
     e2e_ms = sharding.max_over_ranks(e0.elapsed_time(e1), device=dev)
     if world > 1:
         dist.barrier()
-    h2d = x.numel() * x.element_size()
     d2h = qh.numel() + 4 * sh.numel() + 4 * zh.numel()
+    del xh, qh, sh, zh, wsb
+
+    # companion workloads, same kernel family, device-timed the same way (one line, extra keys)
+    companions = {}
+    for ci in args.also:
+        if ci == args.config:
+            continue
+        mc = measure_kernel(torch, sr, syn.workload(ci), args, dev, world, rank, args.quant)
+        del mc["x"]
+        companions[ci] = mc
 
     if rank == 0:
-        bpt = bytes_per_token(w, args.quant)
-        bytes_per_launch = bpt * T
-        avg_launch_ms = region_ms / K  # the fused kernel is the only launch in the region
-        achieved = bytes_per_launch / (avg_launch_ms * 1e-3) / 1e9
         peaks = measured_peaks()
         digest = kernel_sources_digest()
-        traffic = recorded_traffic(w, digest) if args.quant == "asym4" else None
-        value = sharding.aggregate_rate(world * T * K, region_ms_max * 1e-3)
+        K = args.steps
+        value = sharding.aggregate_rate(world * T * K, m["region_ms_max"] * 1e-3)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "ms_per_step": region_ms_max / K, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": m["region_ms_max"] / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {
                 "workload": w.name, "n": n, "tokens_per_gpu": T, "global_tokens": world * T,
@@ -385,28 +466,36 @@ def run_ours(args) -> int:
                            "sym4": "signed INT4 packed [T, n/2] + fp32 scale [T]",
                            "sym8": "int8 [T, n] + fp32 scale [T]"}[args.quant],
                 "parallelism": f"token-sharded x{world} (no collective)",
-                "l2": f"inputs larger than L2 ({bytes_per_launch / 1e6:.1f} MB per step vs "
-                      f"{L2_BYTES / 1e6:.0f} MB), no flush",
+                "l2": l2_note(m),
             },
-            "hbm_gbs": achieved,
-            "hbm_frac": achieved / peaks["hbm_gbs"],
-            "roofline": {
-                "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                "peak_source": peaks["source"], "bytes_per_token": bpt,
-                "kernel": "signrot_rotate_quant" if not sym else "signrot_rotate_quant_sym",
-                "kernel_sources": digest,
-                "launch_ms_mean": avg_launch_ms,
-            },
+            "hbm_gbs": m["achieved"],
+            "hbm_frac": m["achieved"] / peaks["hbm_gbs"],
+            "roofline": roofline_entry(m, args.quant, peaks, digest),
             "e2e": {"value": world * T * E / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / E, "steps": E,
                     "call": "signrot_rotate_quant_host (asymmetric INT4 grid)"},
-            "gpu_launches": int(launches),
-            "calibration": {"tokens": int(xc_np.shape[0]), "ms": calib_ms,
-                            "gbs": xc_np.shape[0] * n * w.in_bytes / (calib_ms * 1e-3) / 1e9},
-            "clocks": sampler.report(),
+            "gpu_launches": int(m["launches"]),
+            "calibration": {"tokens": m["calib_tokens"], "ms": m["calib_ms"],
+                            "gbs": m["calib_tokens"] * n * w.in_bytes / (m["calib_ms"] * 1e-3) / 1e9},
+            "clocks": m["sampler"].report(),
         }
+        if m["warm_ms"] is not None:
+            line["warm_l2"] = {"value": T * K / (m["warm_ms"] * 1e-3), "unit": UNIT,
+                               "gbs": m["bpt"] * T * K / (m["warm_ms"] * 1e-3) / 1e9}
+        if companions:
+            line["also"] = {}
+            for ci, mc in companions.items():
+                wc = mc["w"]
+                entry = {"workload": wc.name, "n": wc.n, "tokens_per_gpu": wc.T,
+                         "value": world * wc.T * K / (mc["region_ms_max"] * 1e-3), "unit": UNIT,
+                         "ms_per_step": mc["region_ms_max"] / K, "l2": l2_note(mc),
+                         "roofline": roofline_entry(mc, args.quant, peaks, digest),
+                         "gpu_launches": int(mc["launches"]), "clocks": mc["sampler"].report()}
+                if mc["warm_ms"] is not None:
+                    entry["warm_l2"] = {"value": wc.T * K / (mc["warm_ms"] * 1e-3), "unit": UNIT,
+                                        "gbs": mc["bpt"] * wc.T * K / (mc["warm_ms"] * 1e-3) / 1e9}
+                line["also"][wc.name] = entry
         if world == 1 and not args.no_cpu_baseline:
             v, done, el = oracle_sample(w, args.cpu_seconds)
             line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
@@ -581,6 +670,7 @@ def run_sweep(args) -> int:
 
 def main(argv=None) -> int:
     args = parse(argv)
+    _default_also(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_sweep(args) if args.sweep else run_ours(args)

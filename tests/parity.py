@@ -48,12 +48,14 @@ def _half_dist(v: np.ndarray) -> np.ndarray:
     return np.abs(v - np.floor(v) - 0.5)
 
 
-def fp32_rotation_bound(x64: np.ndarray) -> np.ndarray:
-    """Per-token bound on |y_fp32 - y_exact| for the rotation computed in fp32."""
+def fp32_rotation_bound(x64: np.ndarray, acc_eps: float = U32) -> np.ndarray:
+    """Per-token bound on |y_fp32 - y_exact| for the rotation accumulated with unit roundoff
+    acc_eps (2^-24: fp32 sums; 2^-53: the fp64 sums of the generic kernel) and rounded once to
+    fp32 at the end (the max |y| * 2^-24 term check_quant adds)."""
     T, n = x64.shape
     F, M = o.factor_n(n)
     S = int(round(math.log2(M))) + (F - 1) + 2
-    return S * U32 * np.abs(x64).sum(axis=1) / math.sqrt(n)
+    return S * acc_eps * np.abs(x64).sum(axis=1) / math.sqrt(n)
 
 
 def oracle_sign(x64: np.ndarray, d: np.ndarray) -> np.ndarray:
@@ -88,14 +90,15 @@ def decode_codes(q: np.ndarray, T: int, n: int, bits: int = 4, sym: bool = False
 
 def check_quant(q_gpu: np.ndarray, scale_gpu: np.ndarray, zero_gpu: np.ndarray | None, y_ref: np.ndarray,
                 clip: float = 1.0, x64: np.ndarray | None = None, bits: int = 4, sym: bool = False,
-                allow_ill: bool | None = None) -> dict:
+                allow_ill: bool | None = None, acc_eps: float = U32) -> dict:
     """Codes, scale and zero-point against the oracle's grid: asymmetric (codes 0 .. 2^bits - 1,
     fp32 zero-point) or, with sym, symmetric (codes -L .. L, L = 2^(bits-1) - 1, no zero-point).
 
     Without x64 every token is held to the bar as stated; with the input rows, tokens whose fp32
     rotation bound alone exceeds the tie window are checked as ill-conditioned (module doc).
     allow_ill (default: only for n < ILL_MAX_N) says whether such tokens may occur at all: rows of
-    ILL_MAX_N channels or more never leave the stated bar."""
+    ILL_MAX_N channels or more never leave the stated bar. acc_eps is the unit roundoff of the
+    kernel's accumulation (fp32 unless the shape runs on the fp64-accumulating generic kernel)."""
     T, n = y_ref.shape
     y32 = y_ref.astype(np.float32)
     if sym:
@@ -126,7 +129,7 @@ def check_quant(q_gpu: np.ndarray, scale_gpu: np.ndarray, zero_gpu: np.ndarray |
     if x64 is None:
         delta = np.zeros(T)
     else:
-        delta = fp32_rotation_bound(x64) + amax * U32
+        delta = fp32_rotation_bound(x64, acc_eps) + amax * U32
     cond = delta / scale_ref  # the fp32 rotation bound in code units
     ill = cond > TIE_EPS
     well = ~ill
