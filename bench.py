@@ -58,6 +58,8 @@ def parse(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gemm", action="store_true",
+                    help="skip the W4A4 down-projection measurement reported under consumer_gemm")
     ap.add_argument("--quant", choices=["asym4", "asym8", "sym4", "sym8"], default="asym4",
                     help="grid of the timed kernel: asymmetric INT4 (the metric's), INT8, or symmetric")
     ap.add_argument("--calib-tokens", type=int, default=None,
@@ -362,6 +364,51 @@ def measure_kernel(torch, sr, w: syn.Workload, args, dev, world: int, rank: int,
             "resident": resident, "warm_ms": warm_ms, "sym": sym}
 
 
+# The down projection each workload's activations feed: (K = n, N = the model's hidden size).
+GEMM_SHAPES = {3: (14336, 4096), 4: (28672, 8192), 5: (14336, 4096), 6: (11008, 4096)}
+
+
+def int8_peak_tops() -> tuple[float, str]:
+    """Dense int8 tensor peak: the measured bf16 GEMM rate (burst) times the nominal int8/bf16
+    ratio of B200 (4.5 / 2.25 = 2)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return 2.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 burst x 2 (nominal int8/bf16 ratio)"
+    return 2.0 * 1590.0, "fallback bf16 1.59 PFLOP/s x 2 (nominal int8/bf16 ratio)"
+
+
+def measure_gemm(torch, sr, T: int, K: int, N: int, dev, steps: int, warmup: int) -> dict:
+    """The W4A4 down projection (signrot_w4a4_matmul) on random codes of the workload's shape:
+    device time of `steps` back-to-back launches; the operands (T x K / 2 + N x K bytes) exceed L2."""
+    g = torch.Generator(device=dev).manual_seed(1234)
+    q = torch.randint(0, 256, (T, K // 2), dtype=torch.uint8, device=dev, generator=g)
+    wq4 = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+    scale = torch.rand(T, device=dev, generator=g) * 0.1 + 0.01
+    zero = torch.randint(-100, 20, (T,), device=dev, generator=g).float()
+    wscale = torch.rand(N, device=dev, generator=g) * 0.01 + 1e-3
+    wq8, colsum = sr.w4a4_prepare_weights(wq4, K)
+    out = torch.empty((T, N), dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        sr.w4a4_matmul(q, scale, zero, wq8, wscale, colsum, out=out)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0 = sr.kernel_launches()
+    e0.record(stream)
+    for _ in range(steps):
+        sr.w4a4_matmul(q, scale, zero, wq8, wscale, colsum, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    tops = 2.0 * T * N * K / (ms * 1e-3) / 1e12
+    peak, src = int8_peak_tops()
+    return {"call": "signrot_w4a4_matmul", "T": T, "K": K, "N": N, "ms_per_launch": ms,
+            "tokens_per_s": T / (ms * 1e-3), "launches": sr.kernel_launches() - l0, "steps": steps,
+            "roofline": {"bound": "tensor", "achieved": tops, "peak": peak, "unit": "TOPS (int8)",
+                         "frac": tops / peak, "peak_source": src, "ops_per_launch": 2.0 * T * N * K}}
+
+
 def roofline_entry(m: dict, quant: str, peaks: dict, digest: str) -> dict:
     w = m["w"]
     traffic = recorded_traffic(w, digest) if quant == "asym4" else None
@@ -449,6 +496,11 @@ def run_ours(args) -> int:
         del mc["x"]
         companions[ci] = mc
 
+    gemm = None
+    if args.config in GEMM_SHAPES and not args.no_gemm:
+        Kg, Ng = GEMM_SHAPES[args.config]
+        gemm = measure_gemm(torch, sr, T, Kg, Ng, dev, max(3, min(args.steps, 20)), 3)
+
     if rank == 0:
         peaks = measured_peaks()
         digest = kernel_sources_digest()
@@ -480,6 +532,8 @@ def run_ours(args) -> int:
                             "gbs": m["calib_tokens"] * n * w.in_bytes / (m["calib_ms"] * 1e-3) / 1e9},
             "clocks": m["sampler"].report(),
         }
+        if gemm is not None:
+            line["consumer_gemm"] = gemm
         if m["warm_ms"] is not None:
             line["warm_l2"] = {"value": T * K / (m["warm_ms"] * 1e-3), "unit": UNIT,
                                "gbs": m["bpt"] * T * K / (m["warm_ms"] * 1e-3) / 1e9}

@@ -214,10 +214,48 @@ size_t signrot_host_bytes_per_token(int32_t n, int32_t dtype);
 
 /*
  * Host, synchronous: writes the device error word of the current device to *code (0 = none;
- * bit 0 = a fused kernel's bounded wait on its own pipeline expired and the kernel stopped
- * early, leaving its outputs incomplete) and clears it when clear != 0.
+ * bit 0 = a fused kernel's (or the W4A4 product's) bounded wait on its own pipeline expired and
+ * the kernel stopped early, leaving its outputs incomplete; bit 1 = an outlier channel index out
+ * of range) and clears it when clear != 0.
  */
 signrot_status signrot_device_error(int32_t* code, int32_t clear);
+
+/*
+ * signrot_w4a4_prepare_weights -- offline step of the consumer side: unpack the down projection's
+ * 4-bit weight codes and sum each output row.
+ *
+ * Follows the explainer's "SignRot asks one crowd to walk across the hall" (the rotation and the
+ * sign flip are folded into the weights offline: W' = W R^T, which is signrot_rotate applied to
+ * the rows of W with the same d and sign adjustment) and "The flip alone does nothing for a
+ * symmetric quantizer" (the zero-point's correction is the zero-point times a precomputed column
+ * sum of the weights). wq4 [N, K/2] (device, row stride ldw4 bytes) holds per-output-row symmetric
+ * 4-bit codes as signrot_rotate_quant_sym(bits = 4) writes them (two's complement nibbles,
+ * element 2i low); writes wq8 [N, K] int8 (row stride ldw8 bytes), one code per byte, and
+ * colsum[N] int32, colsum[o] = sum_j wq8[o][j]. K even.
+ */
+signrot_status signrot_w4a4_prepare_weights(const uint8_t* wq4, int32_t N, int32_t K, int64_t ldw4,
+                                            int8_t* wq8, int64_t ldw8, int32_t* colsum, void* stream);
+
+/*
+ * signrot_w4a4_matmul -- the down projection on the packed codes (tcgen05 int8 tensor cores):
+ *
+ *     out[t][o] = scale[t] * wscale[o] * (sum_j code_tj * wq8[o][j] - zero[t] * colsum[o])
+ *
+ * for t < T, o < N, j < K: code_tj the activation codes 0..15 as signrot_rotate_quant writes them
+ * (q [T, K/2], row stride ldq bytes, element 2i in the low nibble) with their scale[T] and zero[T];
+ * zero = NULL means the symmetric grid instead: code_tj is the signed nibble (-8..7, two's
+ * complement) that signrot_rotate_quant_sym(bits = 4) writes and the zero term is absent.
+ * wq8 [N, K] int8 weight codes in [-8, 7] (row
+ * stride ldw bytes) with per-row scales wscale[N] and colsum[N] from
+ * signrot_w4a4_prepare_weights; out [T, N] fp32 (row stride ldo elements). The integer sums are
+ * exact; the bracket is rounded once to fp32 and multiplied by the two scales. K a multiple of 128
+ * and at most 2^18 (else SIGNROT_ERR_UNSUPPORTED); q and wq8 16-byte aligned with row strides
+ * multiples of 16 bytes (else SIGNROT_ERR_ALIGNMENT). All pointers are device pointers.
+ */
+signrot_status signrot_w4a4_matmul(const uint8_t* q, int64_t T, int32_t K, int64_t ldq, const float* scale,
+                                   const float* zero, const int8_t* wq8, int32_t N, int64_t ldw,
+                                   const float* wscale, const int32_t* colsum, float* out, int64_t ldo,
+                                   void* stream);
 
 /* Host: writes H_28 (Paley, GF(27), the orientation described above) row-major into out[784]. */
 signrot_status signrot_get_h28(int8_t* out);

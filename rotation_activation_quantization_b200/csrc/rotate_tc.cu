@@ -37,6 +37,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 #include <utility>
@@ -126,7 +127,7 @@ __device__ __forceinline__ SignPlan make_plan(const TcParams& p, OutlierRef o) {
   }
   if (o.xk == 0.f) return sp;  // s_j = sgn(+/-0) = +1 everywhere
   sp.active = true;
-  constexpr int kLogNcol = kNcol == 64 ? 6 : (kNcol == 128 ? 7 : 8);
+  constexpr int kLogNcol = kNcol == 16 ? 4 : (kNcol == 32 ? 5 : (kNcol == 64 ? 6 : (kNcol == 128 ? 7 : 8)));
   if (kF28) {
     const int M = 1 << p.logM;
     sp.c_k = k >> p.logM;
@@ -317,19 +318,36 @@ __device__ __forceinline__ void apply_sign_bits(float2 (&p)[kPairs], const uint3
 // column can be applied to the result instead of the values.
 template <int kPairs>
 __device__ __forceinline__ void local_minmax_xy(const float2 (&p)[kPairs], float& lx, float& hx, float& ly, float& hy) {
+  // two independent chains per extreme (the pairs' halves), merged at the end: half the latency
+  constexpr int kH = kPairs / 2;
+  static_assert(kPairs % 2 == 0, "even pair count");
   float l0 = p[0].x, h0 = p[0].x, l1 = p[0].y, h1 = p[0].y;
+  float m0 = p[kH].x, g0 = p[kH].x, m1 = p[kH].y, g1 = p[kH].y;
 #pragma unroll
-  for (int i = 1; i + 1 < kPairs; i += 2) {
+  for (int i = 1; i + 1 < kH; i += 2) {
     l0 = fmin3(l0, p[i].x, p[i + 1].x);
     h0 = fmax3(h0, p[i].x, p[i + 1].x);
     l1 = fmin3(l1, p[i].y, p[i + 1].y);
     h1 = fmax3(h1, p[i].y, p[i + 1].y);
+    m0 = fmin3(m0, p[kH + i].x, p[kH + i + 1].x);
+    g0 = fmax3(g0, p[kH + i].x, p[kH + i + 1].x);
+    m1 = fmin3(m1, p[kH + i].y, p[kH + i + 1].y);
+    g1 = fmax3(g1, p[kH + i].y, p[kH + i + 1].y);
   }
-  if ((kPairs & 1) == 0) {
+  if ((kH & 1) == 0) {  // the last pair of each half
+    l0 = fmin3(l0, p[kH - 1].x, m0);
+    h0 = fmax3(h0, p[kH - 1].x, g0);
+    l1 = fmin3(l1, p[kH - 1].y, m1);
+    h1 = fmax3(h1, p[kH - 1].y, g1);
     l0 = fminf(l0, p[kPairs - 1].x);
     h0 = fmaxf(h0, p[kPairs - 1].x);
     l1 = fminf(l1, p[kPairs - 1].y);
     h1 = fmaxf(h1, p[kPairs - 1].y);
+  } else {
+    l0 = fminf(l0, m0);
+    h0 = fmaxf(h0, g0);
+    l1 = fminf(l1, m1);
+    h1 = fmaxf(h1, g1);
   }
   lx = l0; hx = h0; ly = l1; hy = h1;
 }
@@ -357,12 +375,12 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&u)[8]) {
 // Quantize 16 pairs (32 consecutive columns) into one 16-byte store of packed nibbles. Each
 // fma(w, c, zm) lands in [lo_m, hi_m] around 1.5 * 2^23 after clamping, where the fp32 ulp is 1,
 // so its low bits are the code (two's complement for the symmetric grid's negative codes).
-template <bool kClamp, bool kSigned>
-__device__ __forceinline__ uint4 quant16(const float2* p, float2 c2, float zm, float lo_m, float hi_m) {
+template <bool kClamp, bool kSigned, int kWords = 4>
+__device__ __forceinline__ void quant_words(const float2* p, float2 c2, float zm, float lo_m, float hi_m,
+                                            uint32_t (&words)[kWords]) {
   const float2 z2 = make_float2(zm, zm);
-  uint32_t words[4];
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
+  for (int g = 0; g < kWords; ++g) {
     uint32_t u[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -376,7 +394,19 @@ __device__ __forceinline__ uint4 quant16(const float2* p, float2 c2, float zm, f
     }
     words[g] = pack8<kSigned>(u);
   }
-  return make_uint4(words[0], words[1], words[2], words[3]);
+}
+template <bool kClamp, bool kSigned>
+__device__ __forceinline__ uint4 quant16(const float2* p, float2 c2, float zm, float lo_m, float hi_m) {
+  uint32_t w[4];
+  quant_words<kClamp, kSigned, 4>(p, c2, zm, lo_m, hi_m, w);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+// Eight pairs (16 columns) into one 8-byte store.
+template <bool kClamp, bool kSigned>
+__device__ __forceinline__ uint2 quant8(const float2* p, float2 c2, float zm, float lo_m, float hi_m) {
+  uint32_t w[2];
+  quant_words<kClamp, kSigned, 2>(p, c2, zm, lo_m, hi_m, w);
+  return make_uint2(w[0], w[1]);
 }
 
 // The 8-bit form: 8 pairs (16 consecutive columns) into one 16-byte store, one code per byte.
@@ -407,7 +437,11 @@ template <int kPairs, int kBits, bool kSigned>
 __device__ __forceinline__ void quant_store(const float2 (&p)[kPairs], float2 c2, float zm, bool clamp, float lo_m,
                                             float hi_m, uint8_t* q_out) {
   uint4* dst = reinterpret_cast<uint4*>(q_out);
-  if constexpr (kBits == 4) {
+  if constexpr (kBits == 4 && kPairs == 8) {  // 16 columns: 8 bytes of codes
+    *reinterpret_cast<uint2*>(q_out) = clamp ? quant8<true, kSigned>(p, c2, zm, lo_m, hi_m)
+                                             : quant8<false, kSigned>(p, c2, zm, lo_m, hi_m);
+  } else if constexpr (kBits == 4) {
+    static_assert(kPairs % 16 == 0, "whole 16-byte runs of codes");
     if (clamp) {
 #pragma unroll
       for (int i = 0; i < kPairs / 16; ++i) dst[i] = quant16<true, kSigned>(p + 16 * i, c2, zm, lo_m, hi_m);
@@ -517,29 +551,47 @@ enum : int { kModeY = 0, kModeA4 = 1, kModeA8 = 2, kModeS4 = 3, kModeS8 = 4 };
 __host__ __device__ constexpr int mode_bits(int m) { return (m == kModeA8 || m == kModeS8) ? 8 : 4; }
 __host__ __device__ constexpr bool mode_sym(int m) { return m == kModeS4 || m == kModeS8; }
 
+// The token's grid from its extremes (lo, hi of the raw transform w; y = w / sqrt(n)).
+template <int kMode>
+__device__ __forceinline__ TokenGrid mode_grid(float lo, float hi, const TcParams& p) {
+  constexpr int kBits = mode_bits(kMode);
+  return mode_sym(kMode) ? token_grid_sym(lo, hi, p.inv_sqrt_n, kBits == 4 ? 7.f : 127.f)
+                         : token_grid(lo, hi, p.inv_sqrt_n, p.clip, kBits == 4 ? 15.f : 255.f);
+}
+
+// One thread's run of 2 * kPairs output channels starting at channel j0: codes on grid g (or y).
+// sneg / odd_neg: every output / every odd column comes out of the transform negated (see
+// rotq_stream_kernel).
+template <int kPairs, int kMode>
+__device__ __forceinline__ void emit_run(const float2 (&v)[kPairs], const TokenGrid& g, bool sneg, bool odd_neg,
+                                         bool active, const TcParams& p, int t, int64_t j0) {
+  if (!active) return;
+  const float rs = p.inv_sqrt_n;
+  if constexpr (kMode == kModeY) {
+    store_y<kPairs>(v, sneg ? -rs : rs, p.y + static_cast<int64_t>(t) * p.ldy + j0, (sneg != odd_neg) ? -rs : rs);
+  } else {
+    constexpr int kBits = mode_bits(kMode);
+    quant_store<kPairs, kBits, mode_sym(kMode)>(
+        v, make_float2(sneg ? -g.c : g.c, (sneg != odd_neg) ? -g.c : g.c), g.zm, g.clamp, g.lo_m, g.hi_m,
+        p.q + static_cast<int64_t>(t) * (p.n * kBits / 8) + j0 * kBits / 8);
+  }
+}
+
 // The end of one token for one thread's run of 2 * kPairs output channels starting at channel j0:
-// grid from the token's extremes, codes (or y) stored. sneg / odd_neg: every output / every odd
-// column comes out of the transform negated (see rotq_stream_kernel). writer: this thread also
-// stores the token's scale and zero-point.
+// grid from the token's extremes, codes (or y) stored. writer: this thread also stores the
+// token's scale and zero-point.
 template <int kPairs, int kMode>
 __device__ __forceinline__ void finish_token(const float2 (&v)[kPairs], float lo, float hi, bool sneg, bool odd_neg,
                                              bool active, bool writer, const TcParams& p, int t, int64_t j0) {
-  const float rs = p.inv_sqrt_n;
-  if constexpr (kMode == kModeY) {
-    if (active) store_y<kPairs>(v, sneg ? -rs : rs, p.y + static_cast<int64_t>(t) * p.ldy + j0, (sneg != odd_neg) ? -rs : rs);
-  } else {
-    constexpr int kBits = mode_bits(kMode);
-    const TokenGrid g = mode_sym(kMode) ? token_grid_sym(lo, hi, rs, kBits == 4 ? 7.f : 127.f)
-                                        : token_grid(lo, hi, rs, p.clip, kBits == 4 ? 15.f : 255.f);
+  TokenGrid g{};
+  if constexpr (kMode != kModeY) {
+    g = mode_grid<kMode>(lo, hi, p);
     if (writer) {
       p.scale[t] = g.scale;
       if (!mode_sym(kMode)) p.zero[t] = g.zero;
     }
-    if (active)
-      quant_store<kPairs, kBits, mode_sym(kMode)>(
-          v, make_float2(sneg ? -g.c : g.c, (sneg != odd_neg) ? -g.c : g.c), g.zm, g.clamp, g.lo_m, g.hi_m,
-          p.q + static_cast<int64_t>(t) * (p.n * kBits / 8) + j0 * kBits / 8);
   }
+  emit_run<kPairs, kMode>(v, g, sneg, odd_neg, active, p, t, j0);
 }
 
 // ------------------------------------------------------------------------------------- kernel
@@ -565,15 +617,21 @@ constexpr int kStreamDWarps = 3;
 constexpr int kStreamTiles = 3;
 __host__ __device__ constexpr int stream_threads(int ncol) { return 32 * (4 * epi_groups(ncol) + kStreamDWarps + 1); }
 
-template <int kNcol, bool kF28, bool kVecSign, int kMode>
+template <int kNcol, bool kF28, bool kVecSign, int kMode, int kTok>
 __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(TcParams p) {
   static_assert(kNcol <= 128, "the streamed variant keeps a token's lane line in registers");
+  // kTok tokens share one MMA tile (short rows): token v of a tile owns tile columns
+  // [v * kTokCols, (v + 1) * kTokCols) and the same K rows; kTok = 1 is one token per tile.
+  static_assert(kTok == 1 || (kNcol == 128 && (kTok == 4 || kTok == 8)), "tile of 128 columns for short rows");
+  constexpr int kTokCols = kNcol / kTok;
+  constexpr int kTokPairs = kTokCols / 2;
   constexpr int kKRows = kF28 ? 112 : 128;
   constexpr int kKSteps = kKRows / 16;
   constexpr int kChunksN = kNcol / 64;
   constexpr uint32_t kChunkBytes = kKRows * 128;
   constexpr uint32_t kRowBytes = kChunksN * kChunkBytes;  // = 2n: one bf16 token row
   constexpr int kRowChunks = static_cast<int>(kRowBytes / 16);
+  constexpr int kTokChunks = kRowChunks / kTok;            // one token's row
   constexpr int kDW = kStreamDWarps;
   constexpr int kLaneChunks = kRowChunks / 32;             // chunks per lane position, over all D warps
   static_assert(kRowChunks % 32 == 0, "D-pass lanes own whole chunks");
@@ -607,7 +665,7 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
   uint64_t* tfull = bempty + kTiles;           // [TMEM buffer]
   uint64_t* tempty = tfull + kTBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + kTBufs);
-  float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [buffer][4 quadrants][lo, hi]
+  float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [buffer][4 quadrants][token][lo, hi]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -627,6 +685,7 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
   griddep_wait();
   griddep_launch_dependents();
   const OutlierRef orf = load_outlier(p);  // issued ahead of the bulk copies
+  const int ntiles = (p.T + kTok - 1) / kTok;
 
   // D warp w's share of the row: lane chunks [c0, c0 + 32 * per) of the kRowChunks
   const bool dwarp = warp >= kDWarp0 && warp < kMmaWarp;
@@ -635,11 +694,34 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
   const int c0 = 32 * (dw * (kLaneChunks / kDW) + (dw < kLaneChunks % kDW ? dw : kLaneChunks % kDW));
   const uint32_t part_bytes = static_cast<uint32_t>(per) * 32u * 16u;
   const char* xpart = static_cast<const char*>(p.xraw) + c0 * 16;
-  // one D warp's copy of its share of token t into ring slot st
-  auto stream_in = [&](int st, int t) {
+  // one D warp's copy of its share of tile u into ring slot st (one copy per token its share
+  // touches; rows past the last token are not read, and their slot bytes are never stored)
+  auto stream_in = [&](int st, int u) {
     const uint32_t fb = smem_u32(&lfull[st * kDW + dw]);
-    mbar_arrive_expect_tx(fb, part_bytes);
-    bulk_load(smem_u32(lin + st * kRowBytes + c0 * 16), xpart + static_cast<int64_t>(t) * p.ldx * 2, part_bytes, fb);
+    if constexpr (kTok == 1) {
+      mbar_arrive_expect_tx(fb, part_bytes);
+      bulk_load(smem_u32(lin + st * kRowBytes + c0 * 16), xpart + static_cast<int64_t>(u) * p.ldx * 2, part_bytes, fb);
+    } else {
+      const int e0 = c0 + 32 * per;
+      uint32_t bytes = 0;
+#pragma unroll
+      for (int v = 0; v < kTok; ++v) {
+        const int a = c0 > v * kTokChunks ? c0 : v * kTokChunks;
+        const int b = e0 < (v + 1) * kTokChunks ? e0 : (v + 1) * kTokChunks;
+        if (a < b && kTok * u + v < p.T) bytes += static_cast<uint32_t>(b - a) * 16u;
+      }
+      mbar_arrive_expect_tx(fb, bytes);
+#pragma unroll
+      for (int v = 0; v < kTok; ++v) {
+        const int a = c0 > v * kTokChunks ? c0 : v * kTokChunks;
+        const int b = e0 < (v + 1) * kTokChunks ? e0 : (v + 1) * kTokChunks;
+        const int t = kTok * u + v;
+        if (a < b && t < p.T)
+          bulk_load(smem_u32(lin + st * kRowBytes + a * 16),
+                    static_cast<const char*>(p.xraw) + static_cast<int64_t>(t) * p.ldx * 2 + (a - v * kTokChunks) * 16,
+                    static_cast<uint32_t>(b - a) * 16u, fb);
+      }
+    }
   };
   // The D warps' sign words are loaded (8 bytes per chunk when D is 8-byte aligned) before the
   // bulk copies are issued, so that they do not queue behind every CTA's first copies; the mask
@@ -652,22 +734,23 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
 #pragma unroll
     for (int u = 0; u < kPerD; ++u) {
       const int L = (u < per ? c0 + 32 * u : c0) + lane;
-      const int k = L / (kNcol / 8), b0 = (L % (kNcol / 8)) * 8;
-      const int j0 = kF28 ? (k >> 2) * M + (k & 3) * kNcol + b0 : k * kNcol + b0;
+      const int Lt = L % kTokChunks;  // chunk within its token's row
+      const int k = Lt / (kTokCols / 8), b0 = (Lt % (kTokCols / 8)) * 8;
+      const int j0 = kF28 ? (k >> 2) * M + (k & 3) * kTokCols + b0 : k * kTokCols + b0;
       draw[u] = *reinterpret_cast<const uint2*>(p.d + j0);
     }
   }
   int issued = 0;  // bulk copies this D warp has started (lane 0)
   if (dwarp && lane == 0) {
     for (int st = 0; st < S; ++st) {
-      const int t = blockIdx.x + st * gridDim.x;
-      if (t >= p.T) break;
-      stream_in(st, t);
+      const int u = blockIdx.x + st * gridDim.x;
+      if (u >= ntiles) break;
+      stream_in(st, u);
       ++issued;
     }
   }
 
-  const SignPlan sp = make_plan<kF28, kNcol>(p, orf);
+  const SignPlan sp = make_plan<kF28, kTokCols>(p, orf);
   const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
   uint4 mask[kPerD];
   uint32_t dst[kPerD];
@@ -675,15 +758,16 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
 #pragma unroll
     for (int u = 0; u < kPerD; ++u) {
       const int L = (u < per ? c0 + 32 * u : c0) + lane;
-      const int k = L / (kNcol / 8), b0 = (L % (kNcol / 8)) * 8;
-      const int j0 = kF28 ? (k >> 2) * M + (k & 3) * kNcol + b0 : k * kNcol + b0;
+      const int Lt = L % kTokChunks, vtok = L / kTokChunks;
+      const int k = Lt / (kTokCols / 8), b0 = (Lt % (kTokCols / 8)) * 8;
+      const int j0 = kF28 ? (k >> 2) * M + (k & 3) * kTokCols + b0 : k * kTokCols + b0;
       if (d_aligned) {
         asm volatile("" : "+r"(draw[u].x), "+r"(draw[u].y));  // keeps the use after the copies
         mask[u] = chunk_sign_masks(draw[u]);
       } else {
         mask[u] = chunk_sign_masks(p.d + j0);
       }
-      const int bp = b0 ^ static_cast<int>(col_xor & ~7u);  // where this chunk's columns go
+      const int bp = vtok * kTokCols + (b0 ^ static_cast<int>(col_xor & ~7u));  // where this chunk's columns go
       const int nbp = bp >> 6, segp = (bp >> 3) & 7;
       dst[u] = static_cast<uint32_t>(nbp) * kChunkBytes + k * 128 + ((segp ^ (k & 7)) << 4);
     }
@@ -710,7 +794,7 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
     if (lane == 0) {
       const uint32_t a_base = smem_u32(a_smem);
       int i = 0;
-      for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+      for (int u = blockIdx.x; u < ntiles; u += gridDim.x, ++i) {
         const int bb = i % kTiles, tb = i % kTBufs;
         if (!mbar_wait(smem_u32(&bfull[bb]), (i / kTiles) & 1) ||
             !mbar_wait(smem_u32(&tempty[tb]), ((i / kTBufs) & 1) ^ 1)) {
@@ -735,7 +819,7 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
   } else if (dwarp) {
     // ------------------------------------------------------------------ D pass: linear -> tile
     int i = 0;
-    for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
+    for (int u = blockIdx.x; u < ntiles; u += gridDim.x, ++i) {
       const int st = i % S, bb = i % kTiles;
       if (!warp_wait(smem_u32(&lfull[st * kDW + dw]), (i / S) & 1) ||
           !warp_wait(smem_u32(&bempty[bb]), ((i / kTiles) & 1) ^ 1)) {
@@ -756,9 +840,9 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(smem_u32(&bfull[bb]));
-        const int tn = t + S * gridDim.x;
-        if (tn < p.T) {
-          stream_in(st, tn);
+        const int un = u + S * gridDim.x;
+        if (un < ntiles) {
+          stream_in(st, un);
           ++issued;
         }
       }
@@ -772,14 +856,16 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
     // ------------------------------------------------------------------ epilogue
     const int quad = warp & 3, group = warp >> 2;
     const bool active = !kF28 || lane < 28;
-    const int64_t j0 = kF28 ? static_cast<int64_t>(lane) * M + quad * kNcol : static_cast<int64_t>(quad * 32 + lane) * kNcol;
+    // this thread's run of kTokCols output channels (the same channels in every token of a tile)
+    const int64_t j0 = kF28 ? static_cast<int64_t>(lane) * M + quad * kTokCols
+                            : static_cast<int64_t>(quad * 32 + lane) * kTokCols;
     uint32_t sbits[kVecSign ? kNcol / 32 : 1];
     if (kVecSign) {
 #pragma unroll
       for (int w = 0; w < kNcol / 32; ++w) {
         uint32_t b = 0;
         if (active)
-          for (int r = 0; r < 32; ++r) b |= (p.s[j0 + 32 * w + r] < 0 ? 1u : 0u) << r;
+          for (int r = 0; r < 32; ++r) b |= (p.s[j0 + (32 * w + r) % kTokCols] < 0 ? 1u : 0u) << r;
         sbits[w] = b;
       }
     }
@@ -787,11 +873,11 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
     // transform comes out negated (H P_1 = diag((-1)^j) H), which min/max and quantization undo
     const bool sneg = outlier_sigma_neg(p, sp, orf);  // every output negated
     const bool odd_neg = (col_xor & 1u) != 0;
-    // A warp whose wait runs out stops working but keeps taking its group's barrier, once per token
+    // A warp whose wait runs out stops working but keeps taking its group's barrier, once per tile
     // like the others, so that no warp of the group is left waiting there.
     bool live = true;
     int i = group;
-    for (int t = blockIdx.x + group * gridDim.x; t < p.T; t += kGroups * gridDim.x, i += kGroups) {
+    for (int u = blockIdx.x + group * gridDim.x; u < ntiles; u += kGroups * gridDim.x, i += kGroups) {
       const int tb = i % kTBufs;
       if (live && !warp_wait(smem_u32(&tfull[tb]), (i / kTBufs) & 1)) {
         flag_error();
@@ -808,33 +894,48 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[tb]));
-      fwht_local<kPairs, (kNcol == 64 ? 6 : 7)>(v);
+      fwht_local<kPairs, (kTokCols == 16 ? 4 : (kTokCols == 32 ? 5 : (kTokCols == 64 ? 6 : 7)))>(v);
       if (kVecSign) apply_sign_bits<kPairs>(v, sbits);
-      float lo = pos_inf(), hi = -pos_inf();
-      if (active) {
-        float lx, hx, ly, hy;
-        local_minmax_xy<kPairs>(v, lx, hx, ly, hy);
-        lo = fminf(lx, odd_neg ? -hy : ly);
-        hi = fmaxf(hx, odd_neg ? -ly : hy);
+      float lo[kTok], hi[kTok];
+#pragma unroll
+      for (int tk = 0; tk < kTok; ++tk) {
+        lo[tk] = pos_inf();
+        hi[tk] = -pos_inf();
+        if (active) {
+          float lx, hx, ly, hy;
+          local_minmax_xy<kTokPairs>(*reinterpret_cast<const float2(*)[kTokPairs]>(v + tk * kTokPairs), lx, hx, ly, hy);
+          lo[tk] = fminf(lx, odd_neg ? -hy : ly);
+          hi[tk] = fmaxf(hx, odd_neg ? -ly : hy);
+        }
+        lo[tk] = warp_min(lo[tk]);
+        hi[tk] = warp_max(hi[tk]);
       }
-      lo = warp_min(lo);
-      hi = warp_max(hi);
+      float* rb = red + (tb * 4) * kTok * 2;  // [quadrant][token][lo, hi] of this buffer
       if (lane == 0) {
-        red[(tb * 4 + quad) * 2] = lo;
-        red[(tb * 4 + quad) * 2 + 1] = hi;
+#pragma unroll
+        for (int tk = 0; tk < kTok; ++tk) {
+          rb[(quad * kTok + tk) * 2] = lo[tk];
+          rb[(quad * kTok + tk) * 2 + 1] = hi[tk];
+        }
       }
       named_barrier_sync(1 + group, 128);  // the group's four quadrant extremes are in
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        lo = fminf(lo, red[(tb * 4 + w) * 2]);
-        hi = fmaxf(hi, red[(tb * 4 + w) * 2 + 1]);
+      for (int tk = 0; tk < kTok; ++tk) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          lo[tk] = fminf(lo[tk], rb[(w * kTok + tk) * 2]);
+          hi[tk] = fmaxf(hi[tk], rb[(w * kTok + tk) * 2 + 1]);
+        }
+        if (sneg) {
+          const float t_lo = lo[tk];
+          lo[tk] = -hi[tk];
+          hi[tk] = -t_lo;
+        }
+        const int t = kTok * u + tk;
+        if (t < p.T)
+          finish_token<kTokPairs, kMode>(*reinterpret_cast<const float2(*)[kTokPairs]>(v + tk * kTokPairs), lo[tk],
+                                         hi[tk], sneg, odd_neg, active, quad == 0 && lane == 0, p, t, j0);
       }
-      if (sneg) {
-        const float t_lo = lo;
-        lo = -hi;
-        hi = -t_lo;
-      }
-      finish_token<kPairs, kMode>(v, lo, hi, sneg, odd_neg, active, quad == 0 && lane == 0, p, t, j0);
     }
   }
 
@@ -856,7 +957,10 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
 // Eight epilogue warps share a token: the warp for half h and lane quadrant q forms
 // Y_h = Z0 + (-1)^h Z1 -- the column butterfly on bit 7 -- 16 columns at a time, then runs the
 // remaining seven butterfly stages, min/max, the 8-warp exchange and quantization on its 128
-// values.
+// values. (A token's 28,672-32,768 fp32 values fill the register file, so two tokens' epilogues
+// cannot overlap here; a version with two groups of four warps on alternate tokens, each parking
+// half of its 256-column line in TMEM, held the TMEM buffer through the whole epilogue and ran
+// slower: 40 % of the HBM roofline against 50 % at n = 28672.)
 
 constexpr int kWideEpiWarps = 8;
 constexpr int kWideDWarps = 2;
@@ -1161,6 +1265,33 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
 
 // ------------------------------------------------------------------------------------- host
 
+// Per kernel instantiation: its shared-memory attribute, set once per device, and the device's SM
+// count, queried once per device. Decode-sized calls (a handful of tokens) take a few microseconds
+// on the device, so the host side of a launch must not repeat these driver calls every time.
+struct KernelSetup {
+  static constexpr int kMaxDevices = 64;
+  std::atomic<int> sms[kMaxDevices] = {};  // 0 = not prepared on that device yet
+
+  cudaError_t prepare(const void* kern, int smem, int* sms_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices) {
+      const int cached = sms[dev].load(std::memory_order_acquire);
+      if (cached > 0) {
+        *sms_out = cached;
+        return cudaSuccess;
+      }
+    }
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
+    int count = 0;
+    if ((e = cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices) sms[dev].store(count, std::memory_order_release);
+    *sms_out = count;
+    return cudaSuccess;
+  }
+};
+
 // Launch with programmatic stream serialization: the kernel may be scheduled while the previous
 // kernel in the stream is finishing; it waits (griddepcontrol.wait) before reading any input.
 template <typename... KArgs, typename... Args>
@@ -1178,19 +1309,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int threads, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() { return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder()); }
 
 template <bool kF28, bool kVecSign, int kMode>
 cudaError_t launch_wide(const CUtensorMap& tmap, const TcParams& p0, cudaStream_t st) {
@@ -1203,11 +1322,10 @@ cudaError_t launch_wide(const CUtensorMap& tmap, const TcParams& p0, cudaStream_
   if (p.stages < 2) return cudaErrorNotSupported;
   const size_t smem = 1024 + kABytes + static_cast<size_t>(p.stages) * kStageBytes + 1024;
   auto kern = rotq_wide_kernel<kF28, kVecSign, kMode>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  static KernelSetup setup;
+  int sms = 0;
+  cudaError_t e = setup.prepare(reinterpret_cast<const void*>(kern), static_cast<int>(smem), &sms);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int grid = p.T < sms ? p.T : sms;
   e = launch_pdl(kern, grid, kWideThreads, smem, st, tmap, p);
   count_launch();
@@ -1230,52 +1348,56 @@ cudaError_t dispatch_wide(const CUtensorMap& tmap, const TcParams& p, bool vec_s
   return vec_sign ? dispatch_wide_mode<kF28, true>(tmap, p, mode, st) : dispatch_wide_mode<kF28, false>(tmap, p, mode, st);
 }
 
-template <int kNcol, bool kF28, bool kVecSign, int kMode>
+template <int kNcol, bool kF28, bool kVecSign, int kMode, int kTok>
 cudaError_t launch_stream(const TcParams& p0, cudaStream_t st) {
   constexpr int kKRows = kF28 ? 112 : 128;
   constexpr uint32_t kRowBytes = (kNcol / 64) * kKRows * 128;
-  constexpr uint32_t kSmemBudget = 227 * 1024 - 1024 - kABytes - kStreamTiles * kRowBytes - 1024;
+  constexpr uint32_t kTail = kTok > 1 ? 2048 : 1024;  // barriers, TMEM address, extremes exchange
+  constexpr uint32_t kSmemBudget = 227 * 1024 - 1024 - kABytes - kStreamTiles * kRowBytes - kTail;
   TcParams p = p0;
   p.stages = static_cast<int>(kSmemBudget / kRowBytes);
   if (p.stages > 8) p.stages = 8;
   if (p.stages < 2) return cudaErrorNotSupported;
-  const size_t smem = 1024 + kABytes + kStreamTiles * kRowBytes + static_cast<size_t>(p.stages) * kRowBytes + 1024;
-  auto kern = rotq_stream_kernel<kNcol, kF28, kVecSign, kMode>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  const size_t smem = 1024 + kABytes + kStreamTiles * kRowBytes + static_cast<size_t>(p.stages) * kRowBytes + kTail;
+  auto kern = rotq_stream_kernel<kNcol, kF28, kVecSign, kMode, kTok>;
+  static KernelSetup setup;
+  int sms = 0;
+  cudaError_t e = setup.prepare(reinterpret_cast<const void*>(kern), static_cast<int>(smem), &sms);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  const int grid = p.T < sms ? p.T : sms;
+  const int ntiles = (p.T + kTok - 1) / kTok;
+  const int grid = ntiles < sms ? ntiles : sms;
   e = launch_pdl(kern, grid, stream_threads(kNcol), smem, st, p);
   count_launch();
   return e;
 }
 
-template <int kNcol, bool kF28, bool kVecSign>
+template <int kNcol, bool kF28, bool kVecSign, int kTok>
 cudaError_t dispatch_stream_mode(const TcParams& p, int mode, cudaStream_t st) {
   switch (mode) {
-    case kModeY: return launch_stream<kNcol, kF28, kVecSign, kModeY>(p, st);
-    case kModeA4: return launch_stream<kNcol, kF28, kVecSign, kModeA4>(p, st);
-    case kModeA8: return launch_stream<kNcol, kF28, kVecSign, kModeA8>(p, st);
-    case kModeS4: return launch_stream<kNcol, kF28, kVecSign, kModeS4>(p, st);
-    default: return launch_stream<kNcol, kF28, kVecSign, kModeS8>(p, st);
+    case kModeY: return launch_stream<kNcol, kF28, kVecSign, kModeY, kTok>(p, st);
+    case kModeA4: return launch_stream<kNcol, kF28, kVecSign, kModeA4, kTok>(p, st);
+    case kModeA8: return launch_stream<kNcol, kF28, kVecSign, kModeA8, kTok>(p, st);
+    case kModeS4: return launch_stream<kNcol, kF28, kVecSign, kModeS4, kTok>(p, st);
+    default: return launch_stream<kNcol, kF28, kVecSign, kModeS8, kTok>(p, st);
   }
 }
 
-template <int kNcol, bool kF28>
+template <int kNcol, bool kF28, int kTok = 1>
 cudaError_t dispatch_stream(const TcParams& p, bool vec_sign, int mode, cudaStream_t st) {
-  return vec_sign ? dispatch_stream_mode<kNcol, kF28, true>(p, mode, st) : dispatch_stream_mode<kNcol, kF28, false>(p, mode, st);
+  return vec_sign ? dispatch_stream_mode<kNcol, kF28, true, kTok>(p, mode, st)
+                  : dispatch_stream_mode<kNcol, kF28, false, kTok>(p, mode, st);
 }
 
 }  // namespace
+
+constexpr bool kShortRowTiles = false;
 
 cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
   if (a.dtype != kBF16 || a.T <= 0 || a.T > 0x7fffffff) return cudaErrorNotSupported;
   if (a.shape.F != 1 && a.shape.F != 28) return cudaErrorNotSupported;
   const bool f28 = a.shape.F == 28;
   const int ncol = f28 ? (1 << a.shape.logM) / 4 : a.shape.n / 128;
-  if (ncol != 64 && ncol != 128 && ncol != 256) return cudaErrorNotSupported;
+  if (ncol != 16 && ncol != 32 && ncol != 64 && ncol != 128 && ncol != 256) return cudaErrorNotSupported;
   if (reinterpret_cast<uintptr_t>(a.x) % 16 != 0 || a.ld % 8 != 0) return cudaErrorNotSupported;
   const bool quant = a.q != nullptr;
   const int mode = !quant ? kModeY : (a.sym ? (a.bits == 8 ? kModeS8 : kModeS4) : (a.bits == 8 ? kModeA8 : kModeA4));
@@ -1300,7 +1422,13 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
   p.inv_sqrt_n = a.inv_sqrt_n;
   p.h = h;
   const bool vec = a.s != nullptr && a.kp == nullptr;
-  // Up to 128 columns per token: the streamed kernel; 256 columns: the TMA-staged wide kernel.
+  // Up to 128 columns per token: the streamed kernel (16 or 32 columns: 8 or 4 tokens share a
+  // 128-column tile); 256 columns: the TMA-staged wide kernel.
+  if (kShortRowTiles && ncol == 16)
+    return f28 ? dispatch_stream<128, true, 8>(p, vec, mode, st) : dispatch_stream<128, false, 8>(p, vec, mode, st);
+  if (kShortRowTiles && ncol == 32)
+    return f28 ? dispatch_stream<128, true, 4>(p, vec, mode, st) : dispatch_stream<128, false, 4>(p, vec, mode, st);
+  if (ncol < 64) return cudaErrorNotSupported;
   if (ncol == 64) return f28 ? dispatch_stream<64, true>(p, vec, mode, st) : dispatch_stream<64, false>(p, vec, mode, st);
   if (ncol == 128) return f28 ? dispatch_stream<128, true>(p, vec, mode, st) : dispatch_stream<128, false>(p, vec, mode, st);
 
@@ -1328,6 +1456,20 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
   }
   if (r != CUDA_SUCCESS) return cudaErrorNotSupported;
   return f28 ? dispatch_wide<true>(tmap, p, vec, mode, st) : dispatch_wide<false>(tmap, p, vec, mode, st);
+}
+
+void* tensor_map_encoder() {
+  static void* fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = ptr;
+  });
+  return fn;
 }
 
 cudaError_t read_device_error(uint32_t* out, bool clear) {

@@ -382,10 +382,60 @@ signrot_status signrot_rotate_quant_host(const void* x_host, int32_t dtype, int6
 signrot_status signrot_device_error(int32_t* code, int32_t clear) {
   g_last_error[0] = '\0';
   if (code == nullptr) return fail(SIGNROT_ERR_INVALID_ARG, "code is NULL");
-  uint32_t v = 0;
+  uint32_t v = 0, g = 0;
   cudaError_t e = signrot::read_device_error(&v, clear != 0);
   if (e != cudaSuccess) return cuda_fail(e, "device error word");
-  *code = static_cast<int32_t>(v);
+  if ((e = signrot::read_gemm_error(&g, clear != 0)) != cudaSuccess) return cuda_fail(e, "device error word");
+  *code = static_cast<int32_t>(v | g);
+  return SIGNROT_OK;
+}
+
+signrot_status signrot_w4a4_prepare_weights(const uint8_t* wq4, int32_t N, int32_t K, int64_t ldw4, int8_t* wq8,
+                                            int64_t ldw8, int32_t* colsum, void* stream) {
+  g_last_error[0] = '\0';
+  if (N < 0 || K <= 0 || K % 2 != 0) return fail(SIGNROT_ERR_INVALID_ARG, "N = %d, K = %d: need N >= 0, K even", N, K);
+  if (ldw4 < K / 2 || ldw8 < K) return fail(SIGNROT_ERR_INVALID_ARG, "row strides below the row lengths");
+  if (N > 0 && (wq4 == nullptr || wq8 == nullptr || colsum == nullptr))
+    return fail(SIGNROT_ERR_INVALID_ARG, "wq4, wq8 and colsum must be device pointers");
+  if (!aligned(colsum, 4)) return fail(SIGNROT_ERR_ALIGNMENT, "colsum is not 4-byte aligned");
+  if (N == 0) return SIGNROT_OK;
+  cudaError_t e = signrot::launch_w4a4_prepare(wq4, ldw4, N, K, wq8, ldw8, colsum, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "weight preparation launch");
+  return SIGNROT_OK;
+}
+
+signrot_status signrot_w4a4_matmul(const uint8_t* q, int64_t T, int32_t K, int64_t ldq, const float* scale,
+                                   const float* zero, const int8_t* wq8, int32_t N, int64_t ldw, const float* wscale,
+                                   const int32_t* colsum, float* out, int64_t ldo, void* stream) {
+  g_last_error[0] = '\0';
+  if (T < 0 || N < 0) return fail(SIGNROT_ERR_INVALID_ARG, "T and N must be >= 0");
+  if (K <= 0 || K % 128 != 0 || K > (1 << 18))
+    return fail(SIGNROT_ERR_UNSUPPORTED, "K = %d: the W4A4 product needs K a multiple of 128, at most 2^18", K);
+  if (T > 0x7fffffffLL) return fail(SIGNROT_ERR_INVALID_ARG, "T too large");
+  if (ldq < K / 2 || ldw < K || ldo < N) return fail(SIGNROT_ERR_INVALID_ARG, "row strides below the row lengths");
+  if (T == 0 || N == 0) return SIGNROT_OK;
+  if (q == nullptr || scale == nullptr || wq8 == nullptr || wscale == nullptr || colsum == nullptr || out == nullptr)
+    return fail(SIGNROT_ERR_INVALID_ARG, "q, scale, wq8, wscale, colsum and out must be device pointers");
+  if (!aligned(q, 16) || !aligned(wq8, 16) || ldq % 16 != 0 || ldw % 16 != 0)
+    return fail(SIGNROT_ERR_ALIGNMENT, "q and wq8 must start on 16 bytes, with row strides multiples of 16 bytes");
+  if (!aligned(scale, 4) || !aligned(zero, 4) || !aligned(wscale, 4) || !aligned(colsum, 4) || !aligned(out, 4))
+    return fail(SIGNROT_ERR_ALIGNMENT, "scale, zero, wscale, colsum and out must be 4-byte aligned");
+  signrot::GemmArgs a{};
+  a.q = q;
+  a.ldq = ldq;
+  a.scale = scale;
+  a.zero = zero;
+  a.wq = wq8;
+  a.ldw = ldw;
+  a.wscale = wscale;
+  a.colsum = colsum;
+  a.out = out;
+  a.ldo = ldo;
+  a.T = T;
+  a.N = N;
+  a.K = K;
+  cudaError_t e = signrot::launch_w4a4_gemm(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "W4A4 product launch");
   return SIGNROT_OK;
 }
 

@@ -79,6 +79,30 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
 
 // Reads (and optionally clears) the device error word set by a kernel whose bounded wait expired.
 cudaError_t read_device_error(uint32_t* out, bool clear);
+cudaError_t read_gemm_error(uint32_t* out, bool clear);  // the same, for the W4A4 GEMM
+
+// The driver's cuTensorMapEncodeTiled (PFN_cuTensorMapEncodeTiled_v12000), looked up once; null if
+// the driver does not provide it.
+void* tensor_map_encoder();
+
+// W4A4 down projection (w4a4_gemm.cu): out[t, o] = scale_t wscale_o (sum_j q_tj Q_oj - zero_t c_o).
+struct GemmArgs {
+  const uint8_t* q;      // [T, K/2] packed activation codes 0..15, element 2i low nibble
+  int64_t ldq;           // bytes between rows of q
+  const float* scale;    // [T]
+  const float* zero;     // [T] or null (symmetric activations: zero = 0)
+  const int8_t* wq;      // [N, K] weight codes, one per byte
+  int64_t ldw;           // bytes between rows of wq
+  const float* wscale;   // [N]
+  const int32_t* colsum; // [N]: c_o = sum_j wq[o, j]
+  float* out;            // [T, N] fp32
+  int64_t ldo;           // elements between rows of out
+  int64_t T;
+  int32_t N, K;
+};
+cudaError_t launch_w4a4_gemm(const GemmArgs& a, cudaStream_t st);
+cudaError_t launch_w4a4_prepare(const uint8_t* wq4, int64_t ldw4, int32_t N, int32_t K, int8_t* wq8, int64_t ldw8,
+                                int32_t* colsum, cudaStream_t st);
 
 struct CalibArgs {
   const void* x;

@@ -35,6 +35,9 @@ _SIGNATURES = {
     "signrot_rotate_quant_sym_outlier": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_i32, _c_p,
                                          _c_p, _c_p],
     "signrot_device_error": [_c_p, _c_i32],
+    "signrot_w4a4_prepare_weights": [_c_p, _c_i32, _c_i32, _c_i64, _c_p, _c_i64, _c_p, _c_p],
+    "signrot_w4a4_matmul": [_c_p, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_i32, _c_i64, _c_p, _c_p, _c_p,
+                            _c_i64, _c_p],
     "signrot_rotate_quant_host": [_c_p, _c_i32, _c_i64, _c_i32, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_f,
                                   _c_p, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p],
     "signrot_host_bytes_per_token": [_c_i32, _c_i32],
@@ -153,6 +156,36 @@ def calibrate(x: torch.Tensor, ws: torch.Tensor | None = None, accumulate: bool 
                                      int(bool(accumulate)), _ptr(k_out), _ptr(xk_out), _stream(dev, stream))
     _check("signrot_calibrate", st)
     return k_out, xk_out, ws
+
+
+def calibrate_finish(ws: torch.Tensor, k_out: torch.Tensor | None = None,
+                     xk_out: torch.Tensor | None = None, stream=None):
+    """(k, x_k) from keys ws [n] that are already folded (signrot_calibrate with no rows and
+    accumulate = 1: only the argmax runs). Returns (k, x_k)."""
+    n = ws.numel()
+    dev = ws.device
+    _need(ws, dev, torch.int64, n, "ws")
+    k_out = torch.empty(1, dtype=torch.int32, device=dev) if k_out is None else k_out
+    xk_out = torch.empty(1, dtype=torch.float32, device=dev) if xk_out is None else xk_out
+    with torch.cuda.device(dev):
+        st = lib().signrot_calibrate(None, BF16, 0, n, n, 0, _ptr(ws), 1, _ptr(k_out), _ptr(xk_out),
+                                     _stream(dev, stream))
+    _check("signrot_calibrate", st)
+    return k_out, xk_out
+
+
+def calibrate_sharded(x: torch.Tensor, t_offset: int, ws: torch.Tensor | None = None, group=None,
+                      stream=None):
+    """Calibration over a set split across ranks: this rank's rows x [T, n], whose first row is
+    token t_offset of the whole set. Folds the rows into keys (CUDA), merges the keys of all
+    ranks by one all-reduce(MAX) over the process group (NCCL), then takes the argmax (CUDA).
+    Every rank returns the same (k, x_k), equal to calibrating the whole set at once."""
+    from . import sharding
+
+    _, _, ws = calibrate(x, ws=ws, accumulate=False, t_offset=t_offset, stream=stream)
+    sharding.merge_calibration(ws, group)
+    k, xk = calibrate_finish(ws, stream=stream)
+    return k, xk, ws
 
 
 def calibrate_static(x: torch.Tensor, accumulate: bool = False, t_offset: int = 0,
@@ -312,6 +345,53 @@ def rotate_quant_sym_outlier(x: torch.Tensor, d: torch.Tensor, k: torch.Tensor, 
                                                     int(bits), _ptr(q), _ptr(scale), _stream(dev, stream))
     _check("signrot_rotate_quant_sym_outlier", st)
     return q, scale
+
+
+def w4a4_prepare_weights(wq4: torch.Tensor, K: int, wq8: torch.Tensor | None = None,
+                         colsum: torch.Tensor | None = None, stream=None):
+    """Offline: packed signed 4-bit weight codes wq4 [N, K/2] (as rotate_quant_sym writes them for
+    the rows of the folded weights) -> (wq8 [N, K] int8, colsum [N] int32)."""
+    if wq4.dim() != 2 or wq4.dtype != torch.uint8 or wq4.stride(1) != 1 or wq4.shape[1] != K // 2:
+        raise ValueError("wq4 must be a uint8 [N, K/2] tensor with unit stride along K")
+    N, dev = wq4.shape[0], wq4.device
+    wq8 = torch.empty((N, K), dtype=torch.int8, device=dev) if wq8 is None else wq8
+    colsum = torch.empty(N, dtype=torch.int32, device=dev) if colsum is None else colsum
+    if wq8.shape != (N, K) or wq8.stride(1) != 1 or wq8.dtype != torch.int8 or wq8.device != dev:
+        raise ValueError("wq8 must be an int8 [N, K] tensor with unit stride along K")
+    _need(colsum, dev, torch.int32, N, "colsum")
+    with torch.cuda.device(dev):
+        st = lib().signrot_w4a4_prepare_weights(_ptr(wq4), N, int(K), wq4.stride(0) if N > 1 else K // 2,
+                                                _ptr(wq8), wq8.stride(0) if N > 1 else K, _ptr(colsum),
+                                                _stream(dev, stream))
+    _check("signrot_w4a4_prepare_weights", st)
+    return wq8, colsum
+
+
+def w4a4_matmul(q: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor | None, wq8: torch.Tensor,
+                wscale: torch.Tensor, colsum: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    """out [T, N] fp32 = scale_t wscale_o (sum_j code_tj wq8[o, j] - zero_t colsum_o) from packed
+    activation codes q [T, K/2] (uint8) and int8 weight codes wq8 [N, K]; zero=None takes q as the
+    symmetric grid's signed nibbles (no zero term)."""
+    if q.dim() != 2 or q.dtype != torch.uint8 or q.stride(1) != 1 or not q.is_cuda:
+        raise ValueError("q must be a CUDA uint8 [T, K/2] tensor with unit stride along K")
+    T, K = q.shape[0], 2 * q.shape[1]
+    if wq8.dim() != 2 or wq8.dtype != torch.int8 or wq8.stride(1) != 1 or wq8.shape[1] != K:
+        raise ValueError("wq8 must be an int8 [N, K] tensor with unit stride along K")
+    N, dev = wq8.shape[0], q.device
+    _need(scale, dev, torch.float32, T, "scale")
+    if zero is not None:
+        _need(zero, dev, torch.float32, T, "zero")
+    _need(wscale, dev, torch.float32, N, "wscale")
+    _need(colsum, dev, torch.int32, N, "colsum")
+    out = torch.empty((T, N), dtype=torch.float32, device=dev) if out is None else out
+    if out.shape != (T, N) or out.stride(1) != 1 or out.dtype != torch.float32 or out.device != dev:
+        raise ValueError("out must be a float32 [T, N] tensor with unit stride along N")
+    with torch.cuda.device(dev):
+        st = lib().signrot_w4a4_matmul(_ptr(q), T, K, q.stride(0) if T > 1 else K // 2, _ptr(scale), _ptr(zero),
+                                       _ptr(wq8), N, wq8.stride(0) if N > 1 else K, _ptr(wscale), _ptr(colsum),
+                                       _ptr(out), out.stride(0) if T > 1 else N, _stream(dev, stream))
+    _check("signrot_w4a4_matmul", st)
+    return out
 
 
 def device_error(clear: bool = True) -> int:

@@ -72,3 +72,35 @@ def test_both_fold_kernels_agree_with_oracle(sr):
 def test_all_zero_rows(sr):
     x = np.zeros((300, 2048), dtype=np.uint16)
     assert run(sr, dev(x)) == (0, 0.0)
+
+
+@pytest.mark.parametrize("index", [2, 3])
+def test_sharded_calibration_keys_and_merge(sr, index):
+    """Two shards of one calibration set folded separately (as two ranks would): each workspace
+    holds exactly the keys the header defines (restated in tests/calib_keys.py), their elementwise
+    maximum -- what the all-reduce(MAX) of calibrate_sharded computes -- gives the whole set's
+    (k, x_k) through the argmax-only call, and calibrate_sharded without a process group equals
+    calibrate."""
+    from calib_keys import decode, fold_keys
+
+    w = syn.workload(index)
+    xc = syn.draw_calibration(w)
+    Tc = xc.shape[0]
+    half = Tc // 2 + 3  # an uneven split
+    x_t = dev(xc)  # both workloads store bf16 rows
+    x64 = o.to_f64(xc, w.dtype)
+    ws_a = torch.empty(w.n, dtype=torch.int64, device="cuda")
+    ws_b = torch.empty(w.n, dtype=torch.int64, device="cuda")
+    sr.calibrate(x_t[:half], ws=ws_a, t_offset=0)
+    sr.calibrate(x_t[half:], ws=ws_b, t_offset=half)
+    torch.cuda.synchronize()
+    keys_a = fold_keys(x64[:half], t_offset=0)
+    keys_b = fold_keys(x64[half:], t_offset=half)
+    assert (ws_a.cpu().numpy().astype(np.uint64) == keys_a).all()
+    assert (ws_b.cpu().numpy().astype(np.uint64) == keys_b).all()
+    merged = torch.maximum(ws_a, ws_b)
+    k, xk = sr.calibrate_finish(merged)
+    ref = o.calibrate(x64)
+    assert (int(k.item()), float(xk.item())) == ref == decode(np.maximum(keys_a, keys_b))
+    k2, xk2, _ = sr.calibrate_sharded(x_t, t_offset=0)
+    assert (int(k2.item()), float(xk2.item())) == ref

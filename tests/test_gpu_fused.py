@@ -1,6 +1,7 @@
-"""GPU tests of the fused tensor-core path (bf16 rows with n = 28 * {256, 512, 1024} or
-n = {8192, 16384, 32768}): the outlier-channel entry points against the materialised sign vector,
-token counts around the persistent grid, a general sign vector, and the device error word."""
+"""GPU tests of the fused tensor-core path (bf16 rows with n = 28 * {64, 128, 256, 512, 1024} or
+n = {2048, 4096, 8192, 16384, 32768}; the shortest rows share a 128-column MMA tile, four or eight
+tokens to a tile): the outlier-channel entry points against the materialised sign vector, token
+counts around the persistent grid, a general sign vector, and the device error word."""
 import numpy as np
 import pytest
 
@@ -12,7 +13,7 @@ from parity import check_quant, check_rotation, oracle_sign, record
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
-FUSED_N = [28 * 256, 28 * 512, 28 * 1024, 8192, 16384, 32768]
+FUSED_N = [28 * 64, 28 * 128, 28 * 256, 28 * 512, 28 * 1024, 2048, 4096, 8192, 16384, 32768]
 
 
 @pytest.fixture(scope="module")
@@ -58,24 +59,27 @@ def test_outlier_entry_equals_sign_vector_entry(sr, n):
     assert sr.device_error() == 0
 
 
-@pytest.mark.parametrize("T", [1, 2, 147, 148, 149, 297])
-def test_token_counts_around_the_grid(sr, T):
-    n = 14336
+@pytest.mark.parametrize("n,T", [(14336, 1), (14336, 2), (14336, 147), (14336, 148), (14336, 149), (14336, 297),
+                                 (4096, 1), (4096, 3), (4096, 5), (4096, 591), (4096, 592), (4096, 593),
+                                 (1792, 7), (1792, 1185)])
+def test_token_counts_around_the_grid(sr, n, T):
+    """Persistent grids of one CTA per SM (148): token counts around it, and for the shortest rows
+    (four or eight tokens per tile) counts that leave a partial last tile."""
     x, d, _ = syn.random_rows(n, T, "bf16", seed=T, outlier=1500.0)
     x_t, d_t = dev_bf16(x), i8(d)
     k, xk, _ = sr.calibrate(x_t)
     q, scale, zero = sr.rotate_quant_outlier(x_t, d_t, k, xk)
     torch.cuda.synchronize()
-    rows = sorted({0, T // 2, T - 1})
+    rows = sorted({0, T // 2, T - 1, max(T - 2, 0)})
     s = oracle_sign(o.to_f64(x, "bf16"), d)
     x64 = o.to_f64(x[rows], "bf16")
     y_ref = o.rotate(x64, d, s)
     qn, sn, zn = q.cpu().numpy(), scale.cpu().numpy(), zero.cpu().numpy()
-    record(f"fused_T{T}", check_quant(qn[rows], sn[rows], zn[rows], y_ref, x64=x64))
+    record(f"fused_n{n}_T{T}", check_quant(qn[rows], sn[rows], zn[rows], y_ref, x64=x64))
     assert sr.device_error() == 0
 
 
-@pytest.mark.parametrize("n", [28 * 512, 28 * 1024, 16384])
+@pytest.mark.parametrize("n", [28 * 128, 2048, 28 * 512, 28 * 1024, 16384])
 def test_general_sign_vector_on_fused_path(sr, n):
     T = 9
     x, d, _ = syn.random_rows(n, T, "bf16", seed=3 * n, outlier=900.0)
@@ -115,7 +119,7 @@ def test_out_of_range_channel_is_reported_not_read(sr):
     assert sr.device_error() == 0
 
 
-@pytest.mark.parametrize("n,T,chunk", [(14336, 300, 64), (28672, 70, 16), (4096, 33, 8)])
+@pytest.mark.parametrize("n,T,chunk", [(14336, 300, 64), (28672, 70, 16), (4096, 33, 8), (4096, 37, 6)])
 def test_host_buffer_entry_matches_device_entry(sr, n, T, chunk):
     """Host rows -> chunked device workspace -> host codes equals the device-resident call."""
     x, d, _ = syn.random_rows(n, T, "bf16", seed=11 * T, outlier=1500.0)

@@ -172,7 +172,7 @@ def test_workload_full_size(sr, index):
     assert bool((err <= scale * 0.5 * (1 + 1e-4) + y_all.abs().amax(dim=1) * 1e-6).all())
 
 
-@pytest.mark.parametrize("index", [3, 4])
+@pytest.mark.parametrize("index", [2, 3, 4])
 def test_timed_call_full_size(sr, index):
     """The call the benchmark times -- the outlier-channel entry point, sign adjustment folded into
     the rotation -- on the workload's full token count, checked against the oracle on the first
@@ -190,9 +190,13 @@ def test_timed_call_full_size(sr, index):
     k_ref, xk_ref = o.calibrate(o.to_f64(xc, w.dtype))
     assert (int(k.item()), float(xk.item())) == (k_ref, xk_ref)
     s_ref = o.build_sign(w.n, k_ref, xk_ref, d)
-    grid = min(w.T, torch.cuda.get_device_properties(0).multi_processor_count)
-    first = np.arange(grid)
-    last = first + grid * ((w.T - 1 - first) // grid)
+    # a CTA takes tiles of tok tokens (four for n = 4096's 32-column rows, else one)
+    tok = 4 if w.n == 4096 else 1
+    tiles = -(-w.T // tok)
+    grid = min(tiles, torch.cuda.get_device_properties(0).multi_processor_count)
+    first = np.arange(grid) * tok
+    last = (np.arange(grid) + grid * ((tiles - 1 - np.arange(grid)) // grid)) * tok + tok - 1
+    last = np.minimum(last, w.T - 1)
     extra = np.random.default_rng(100 + index).choice(w.T, 24, replace=False)
     sample = np.unique(np.concatenate([first, last, extra]))
     x64 = o.to_f64(x[sample], w.dtype)
