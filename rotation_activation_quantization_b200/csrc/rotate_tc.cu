@@ -318,36 +318,19 @@ __device__ __forceinline__ void apply_sign_bits(float2 (&p)[kPairs], const uint3
 // column can be applied to the result instead of the values.
 template <int kPairs>
 __device__ __forceinline__ void local_minmax_xy(const float2 (&p)[kPairs], float& lx, float& hx, float& ly, float& hy) {
-  // two independent chains per extreme (the pairs' halves), merged at the end: half the latency
-  constexpr int kH = kPairs / 2;
-  static_assert(kPairs % 2 == 0, "even pair count");
   float l0 = p[0].x, h0 = p[0].x, l1 = p[0].y, h1 = p[0].y;
-  float m0 = p[kH].x, g0 = p[kH].x, m1 = p[kH].y, g1 = p[kH].y;
 #pragma unroll
-  for (int i = 1; i + 1 < kH; i += 2) {
+  for (int i = 1; i + 1 < kPairs; i += 2) {
     l0 = fmin3(l0, p[i].x, p[i + 1].x);
     h0 = fmax3(h0, p[i].x, p[i + 1].x);
     l1 = fmin3(l1, p[i].y, p[i + 1].y);
     h1 = fmax3(h1, p[i].y, p[i + 1].y);
-    m0 = fmin3(m0, p[kH + i].x, p[kH + i + 1].x);
-    g0 = fmax3(g0, p[kH + i].x, p[kH + i + 1].x);
-    m1 = fmin3(m1, p[kH + i].y, p[kH + i + 1].y);
-    g1 = fmax3(g1, p[kH + i].y, p[kH + i + 1].y);
   }
-  if ((kH & 1) == 0) {  // the last pair of each half
-    l0 = fmin3(l0, p[kH - 1].x, m0);
-    h0 = fmax3(h0, p[kH - 1].x, g0);
-    l1 = fmin3(l1, p[kH - 1].y, m1);
-    h1 = fmax3(h1, p[kH - 1].y, g1);
+  if ((kPairs & 1) == 0) {
     l0 = fminf(l0, p[kPairs - 1].x);
     h0 = fmaxf(h0, p[kPairs - 1].x);
     l1 = fminf(l1, p[kPairs - 1].y);
     h1 = fmaxf(h1, p[kPairs - 1].y);
-  } else {
-    l0 = fminf(l0, m0);
-    h0 = fmaxf(h0, g0);
-    l1 = fminf(l1, m1);
-    h1 = fmaxf(h1, g1);
   }
   lx = l0; hx = h0; ly = l1; hy = h1;
 }
@@ -622,7 +605,7 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
   static_assert(kNcol <= 128, "the streamed variant keeps a token's lane line in registers");
   // kTok tokens share one MMA tile (short rows): token v of a tile owns tile columns
   // [v * kTokCols, (v + 1) * kTokCols) and the same K rows; kTok = 1 is one token per tile.
-  static_assert(kTok == 1 || (kNcol == 128 && (kTok == 4 || kTok == 8)), "tile of 128 columns for short rows");
+  static_assert(kTok == 1 || (kNcol == 128 && kTok == 4), "tile of 128 columns for short rows");
   constexpr int kTokCols = kNcol / kTok;
   constexpr int kTokPairs = kTokCols / 2;
   constexpr int kKRows = kF28 ? 112 : 128;
@@ -754,6 +737,32 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
   const uint32_t col_xor = sp.active ? sp.e_lo : 0u;
   uint4 mask[kPerD];
   uint32_t dst[kPerD];
+  // Short rows (several tokens per tile) with an outlier plan: the outlier channel k is left out of
+  // the MMA (its element is zeroed in the tile) and its exact contribution, sgn(x_k) x_{t,k} on
+  // every sign-adjusted output, is added once after the butterflies. The massive value then never
+  // passes through the fp32 sums, whose rounding at its magnitude would otherwise move a row's
+  // codes near rounding ties. kill[v]: byte offset in the tile of token v's element k when this
+  // lane writes it, else ~0.
+  // kill, packed: bits 0-15 the element's byte offset in its chunk row (K row * 128 + offset inside
+  // the 16-byte chunk), bits 16-17 the permuted chunk within the token's 32 columns, bits 18-20
+  // the K row's swizzle phase, bits 24+ one bit per token v whose element k this lane writes.
+  uint32_t kill = 0;
+  if (kTok > 1 && dwarp && sp.active) {
+    const int kk = orf.k;
+    const int rk = kF28 ? 4 * (kk >> p.logM) + ((kk & (M - 1)) / kTokCols) : kk / kTokCols;  // K row
+    const int bk = kk % kTokCols;                                                            // input column
+    const int ltk = rk * (kTokCols / 8) + (bk >> 3);                                         // chunk in its row
+    const int kw = static_cast<int>((col_xor >> 1) & 3u), ek = bk & 7;
+    static_assert(kTok == 1 || kTokCols == 32, "packed kill state assumes 32-column tokens");
+#pragma unroll
+    for (int v = 0; v < kTok; ++v) {
+      const int L = v * kTokChunks + ltk;
+      if (L >= c0 && L < c0 + 32 * per && (L - c0) % 32 == lane) kill |= 1u << (24 + v);
+    }
+    const uint32_t col = static_cast<uint32_t>((bk & ~7) ^ static_cast<int>(col_xor & ~7u));  // < 32
+    kill |= static_cast<uint32_t>(rk * 128 + ((((ek >> 1) ^ kw) << 2) | ((ek & 1) << 1))) | ((col >> 3) << 16) |
+            ((static_cast<uint32_t>(rk) & 7u) << 18);
+  }
   if (dwarp) {
 #pragma unroll
     for (int u = 0; u < kPerD; ++u) {
@@ -834,6 +843,17 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
         case 2: stream_d_pass<2, kPerD, kDBatch>(src, tile, mask, dst, last); break;
         default: stream_d_pass<3, kPerD, kDBatch>(src, tile, mask, dst, last); break;
       }
+      if constexpr (kTok > 1) {
+#pragma unroll
+        for (int v = 0; v < kTok; ++v) {
+          if ((kill >> (24 + v)) & 1u) {  // the chunk was written above by this lane
+            // token v's 32 columns start at column 32 v: 64-column block v / 2, 16-byte slot 4 (v % 2)
+            const uint32_t segp = 4u * (v & 1) + ((kill >> 16) & 3u);
+            *reinterpret_cast<uint16_t*>(tile + (v >> 1) * kChunkBytes + (kill & 0xffffu) +
+                                         ((segp ^ ((kill >> 18) & 7u)) << 4)) = 0;
+          }
+        }
+      }
       // the tile writes must reach the MMA (async proxy), and this slot's reads must be done
       // before the next bulk copy overwrites it
       fence_proxy_async_smem();
@@ -896,6 +916,19 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
       if (lane == 0) mbar_arrive(smem_u32(&tempty[tb]));
       fwht_local<kPairs, (kTokCols == 16 ? 4 : (kTokCols == 32 ? 5 : (kTokCols == 64 ? 6 : 7)))>(v);
       if (kVecSign) apply_sign_bits<kPairs>(v, sbits);
+      // short rows: the tokens' outlier values, left out of the MMA (see kill); their contribution
+      // sgn(x_k) x_{t,k} to every sign-adjusted output is added after the extremes are known
+      float dlt[kTok];
+#pragma unroll
+      for (int tk = 0; tk < kTok; ++tk) {
+        const int t = kTok * u + tk;
+        dlt[tk] = 0.f;
+        if (kTok > 1 && sp.active && t < p.T) {
+          const float xv = __uint_as_float(
+              static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(p.xraw)[static_cast<int64_t>(t) * p.ldx + orf.k]) << 16);
+          dlt[tk] = orf.xk < 0.f ? -xv : xv;
+        }
+      }
       float lo[kTok], hi[kTok];
 #pragma unroll
       for (int tk = 0; tk < kTok; ++tk) {
@@ -930,6 +963,14 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
           const float t_lo = lo[tk];
           lo[tk] = -hi[tk];
           hi[tk] = -t_lo;
+        }
+        if constexpr (kTok > 1) {
+          // each output rounds once, RN(v + shift); rounding is monotone, so the extremes shift alike
+          lo[tk] = __fadd_rn(lo[tk], dlt[tk]);
+          hi[tk] = __fadd_rn(hi[tk], dlt[tk]);
+          const float2 d2 = make_float2(sneg ? -dlt[tk] : dlt[tk], (sneg != odd_neg) ? -dlt[tk] : dlt[tk]);
+#pragma unroll
+          for (int i = 0; i < kTokPairs; ++i) v[tk * kTokPairs + i] = __fadd2_rn(v[tk * kTokPairs + i], d2);
         }
         const int t = kTok * u + tk;
         if (t < p.T)
@@ -1390,14 +1431,14 @@ cudaError_t dispatch_stream(const TcParams& p, bool vec_sign, int mode, cudaStre
 
 }  // namespace
 
-constexpr bool kShortRowTiles = false;
+constexpr bool kShortRowTiles = true;
 
 cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
   if (a.dtype != kBF16 || a.T <= 0 || a.T > 0x7fffffff) return cudaErrorNotSupported;
   if (a.shape.F != 1 && a.shape.F != 28) return cudaErrorNotSupported;
   const bool f28 = a.shape.F == 28;
   const int ncol = f28 ? (1 << a.shape.logM) / 4 : a.shape.n / 128;
-  if (ncol != 16 && ncol != 32 && ncol != 64 && ncol != 128 && ncol != 256) return cudaErrorNotSupported;
+  if (ncol != 32 && ncol != 64 && ncol != 128 && ncol != 256) return cudaErrorNotSupported;
   if (reinterpret_cast<uintptr_t>(a.x) % 16 != 0 || a.ld % 8 != 0) return cudaErrorNotSupported;
   const bool quant = a.q != nullptr;
   const int mode = !quant ? kModeY : (a.sym ? (a.bits == 8 ? kModeS8 : kModeS4) : (a.bits == 8 ? kModeA8 : kModeA4));
@@ -1422,10 +1463,13 @@ cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStrea
   p.inv_sqrt_n = a.inv_sqrt_n;
   p.h = h;
   const bool vec = a.s != nullptr && a.kp == nullptr;
-  // Up to 128 columns per token: the streamed kernel (16 or 32 columns: 8 or 4 tokens share a
-  // 128-column tile); 256 columns: the TMA-staged wide kernel.
-  if (kShortRowTiles && ncol == 16)
-    return f28 ? dispatch_stream<128, true, 8>(p, vec, mode, st) : dispatch_stream<128, false, 8>(p, vec, mode, st);
+  // Up to 128 columns per token: the streamed kernel (32 columns: 4 tokens share a 128-column
+  // tile); 256 columns: the TMA-staged wide kernel. Shorter rows take the generic kernel.
+  // Short rows with a materialised sign vector take the generic (exact) kernel: only the outlier
+  // form tells the kernel which channel to keep out of the fp32 sums (see kill in
+  // rotq_stream_kernel), and a sign vector built from the outlier gives exactly the rows (one
+  // crowd far from zero, a narrow spread) where those sums' rounding would reach the codes.
+  if (ncol == 32 && vec) return cudaErrorNotSupported;
   if (kShortRowTiles && ncol == 32)
     return f28 ? dispatch_stream<128, true, 4>(p, vec, mode, st) : dispatch_stream<128, false, 4>(p, vec, mode, st);
   if (ncol < 64) return cudaErrorNotSupported;

@@ -1,5 +1,5 @@
-"""GPU tests of the fused tensor-core path (bf16 rows with n = 28 * {64, 128, 256, 512, 1024} or
-n = {2048, 4096, 8192, 16384, 32768}; the shortest rows share a 128-column MMA tile, four or eight
+"""GPU tests of the fused tensor-core path (bf16 rows with n = 28 * {128, 256, 512, 1024} or
+n = {4096, 8192, 16384, 32768}; the shortest, n = 3584 and 4096, share a 128-column MMA tile four
 tokens to a tile): the outlier-channel entry points against the materialised sign vector, token
 counts around the persistent grid, a general sign vector, and the device error word."""
 import numpy as np
@@ -13,7 +13,7 @@ from parity import check_quant, check_rotation, oracle_sign, record
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
-FUSED_N = [28 * 64, 28 * 128, 28 * 256, 28 * 512, 28 * 1024, 2048, 4096, 8192, 16384, 32768]
+FUSED_N = [28 * 128, 28 * 256, 28 * 512, 28 * 1024, 4096, 8192, 16384, 32768]
 
 
 @pytest.fixture(scope="module")
@@ -35,9 +35,13 @@ def i8(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int8)).cuda()
 
 
+SHORT_N = (28 * 128, 4096)  # four tokens per tile; a sign vector takes the exact generic kernel there
+
+
 @pytest.mark.parametrize("n", FUSED_N)
 def test_outlier_entry_equals_sign_vector_entry(sr, n):
-    """Folding s into the rotation gives the same bits as applying the materialised s."""
+    """Folding s into the rotation gives the same bits as applying the materialised s (on the
+    short rows the two entries run different kernels: each is checked against the oracle)."""
     T = 37
     x, d, _ = syn.random_rows(n, T, "bf16", seed=n, outlier=1800.0)
     x_t, d_t = dev_bf16(x), i8(d)
@@ -45,10 +49,11 @@ def test_outlier_entry_equals_sign_vector_entry(sr, n):
     s_t = sr.build_sign(n, k, xk, d_t)
     q1, s1, z1 = sr.rotate_quant(x_t, d_t, s_t)
     q2, s2, z2 = sr.rotate_quant_outlier(x_t, d_t, k, xk)
-    assert torch.equal(q1, q2) and torch.equal(s1, s2) and torch.equal(z1, z2)
     y1 = sr.rotate(x_t, d_t, s_t)
     y2 = sr.rotate_outlier(x_t, d_t, k, xk)
-    assert torch.equal(y1, y2)
+    if n not in SHORT_N:
+        assert torch.equal(q1, q2) and torch.equal(s1, s2) and torch.equal(z1, z2)
+        assert torch.equal(y1, y2)
     x64 = o.to_f64(x, "bf16")
     s_ref = oracle_sign(x64, d)
     assert (s_t.cpu().numpy() == s_ref).all()
@@ -56,15 +61,18 @@ def test_outlier_entry_equals_sign_vector_entry(sr, n):
     st = check_rotation(y2.cpu().numpy(), y_ref)
     st.update(check_quant(q2.cpu().numpy(), s2.cpu().numpy(), z2.cpu().numpy(), y_ref, x64=x64))
     record(f"fused_outlier_{n}", st)
+    if n in SHORT_N:
+        check_rotation(y1.cpu().numpy(), y_ref)
+        record(f"fused_vector_{n}", check_quant(q1.cpu().numpy(), s1.cpu().numpy(), z1.cpu().numpy(), y_ref, x64=x64))
     assert sr.device_error() == 0
 
 
 @pytest.mark.parametrize("n,T", [(14336, 1), (14336, 2), (14336, 147), (14336, 148), (14336, 149), (14336, 297),
                                  (4096, 1), (4096, 3), (4096, 5), (4096, 591), (4096, 592), (4096, 593),
-                                 (1792, 7), (1792, 1185)])
+                                 (3584, 7), (3584, 1185)])
 def test_token_counts_around_the_grid(sr, n, T):
     """Persistent grids of one CTA per SM (148): token counts around it, and for the shortest rows
-    (four or eight tokens per tile) counts that leave a partial last tile."""
+    (four tokens per tile) counts that leave a partial last tile."""
     x, d, _ = syn.random_rows(n, T, "bf16", seed=T, outlier=1500.0)
     x_t, d_t = dev_bf16(x), i8(d)
     k, xk, _ = sr.calibrate(x_t)
@@ -79,7 +87,7 @@ def test_token_counts_around_the_grid(sr, n, T):
     assert sr.device_error() == 0
 
 
-@pytest.mark.parametrize("n", [28 * 128, 2048, 28 * 512, 28 * 1024, 16384])
+@pytest.mark.parametrize("n", [28 * 128, 4096, 28 * 512, 28 * 1024, 16384])
 def test_general_sign_vector_on_fused_path(sr, n):
     T = 9
     x, d, _ = syn.random_rows(n, T, "bf16", seed=3 * n, outlier=900.0)
@@ -134,10 +142,11 @@ def test_host_buffer_entry_matches_device_entry(sr, n, T, chunk):
     sr.rotate_quant_host(xh, d_t, qh, sh, zh, ws, k=k, xk=xk)
     torch.cuda.synchronize()
     assert torch.equal(qh, q.cpu()) and torch.equal(sh, scale.cpu()) and torch.equal(zh, zero.cpu())
-    # a general sign vector through the same entry
+    # a general sign vector through the same entry equals the device-resident vector call
     s_t = sr.build_sign(n, k, xk, d_t)
+    qv, _, _ = sr.rotate_quant(x_t, d_t, s_t)
     sr.rotate_quant_host(xh, d_t, qh, sh, zh, ws, s=s_t)
     torch.cuda.synchronize()
-    assert torch.equal(qh, q.cpu())
+    assert torch.equal(qh, qv.cpu())
     with pytest.raises(sr.SignRotError):
         sr.rotate_quant_host(xh, d_t, qh, sh, zh, ws[:16], k=k, xk=xk)

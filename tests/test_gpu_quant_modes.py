@@ -51,20 +51,27 @@ def test_quantizer_variants(sr, n, dtype):
     s_ref = oracle_sign(x64, d)
     assert (s_t.cpu().numpy() == s_ref).all()
     y_ref = o.rotate(x64, d, s_ref)
+    # on the short rows (n = 3584, 4096) the two entries run different kernels: each is checked
+    same_kernel = not (dtype == "bf16" and n in (3584, 4096))
     for bits, sym in MODES:
         if sym:
             q1, sc1 = sr.rotate_quant_sym(x_t, d_t, s_t, bits=bits)
             q2, sc2 = sr.rotate_quant_sym_outlier(x_t, d_t, k, xk, bits=bits)
-            z2 = None
-            assert torch.equal(q1, q2) and torch.equal(sc1, sc2)
+            z1 = z2 = None
+            if same_kernel:
+                assert torch.equal(q1, q2) and torch.equal(sc1, sc2)
         else:
             q1, sc1, z1 = sr.rotate_quant(x_t, d_t, s_t, bits=bits)
             q2, sc2, z2 = sr.rotate_quant_outlier(x_t, d_t, k, xk, bits=bits)
-            assert torch.equal(q1, q2) and torch.equal(sc1, sc2) and torch.equal(z1, z2)
+            if same_kernel:
+                assert torch.equal(q1, q2) and torch.equal(sc1, sc2) and torch.equal(z1, z2)
         torch.cuda.synchronize()
         st = check_quant(q2.cpu().numpy(), sc2.cpu().numpy(), None if z2 is None else z2.cpu().numpy(), y_ref,
                          x64=x64, bits=bits, sym=sym)
         record(f"mode_{'sym' if sym else 'asym'}{bits}_{n}", st)
+        if not same_kernel:
+            check_quant(q1.cpu().numpy(), sc1.cpu().numpy(), None if z1 is None else z1.cpu().numpy(), y_ref,
+                        x64=x64, bits=bits, sym=sym)
     assert sr.device_error() == 0
 
 
