@@ -22,12 +22,12 @@
 // one fp32 FMA of exact operands (a single rounding), then the two scales.
 //
 // Tile: 128 tokens x 256 outputs per CTA, K in blocks of 128 bytes (one 128-byte swizzle atom).
-// Warp roles (256 threads, one CTA per SM, persistent over tiles):
+// Warp roles (320 threads, one CTA per SM, persistent over tiles):
 //   warp 0     TMA producer: weight block [256 x 128] (swizzled, straight into the MMA tile) and
 //              packed activation block [128 x 64 bytes]
-//   warps 1-2  converters: packed codes -> the MMA's swizzled s8 activation tile
-//   warp 3     TMEM allocator and MMA issuer (4 x M128 N256 K32 per K block)
-//   warps 4-7  epilogue (TMEM lane quadrant = warp % 4): accumulator -> fp32 outputs
+//   warps 1-4  converters: packed codes -> the MMA's swizzled s8 activation tile
+//   warp 5     TMEM allocator and MMA issuer (4 x M128 N256 K32 per K block)
+//   warps 6-9  epilogue (TMEM lane quadrant = warp % 4): accumulator -> fp32 outputs
 // Pipeline: TMA -> loaded[s] -> convert -> ready[s] -> MMA -> empty[s]; the accumulator is double
 // buffered in TMEM (2 x 256 columns) so one tile's epilogue overlaps the next tile's K loop.
 #include <cuda.h>
@@ -55,8 +55,11 @@ constexpr int kGStages = 4;
 constexpr uint32_t kBBytes = kGN * kGK;      // 32 KB weight block
 constexpr uint32_t kABytes8 = kGM * kGK;     // 16 KB s8 activation block
 constexpr uint32_t kPBytes = kGM * kGK / 2;  // 8 KB packed activation block
-constexpr int kConvWarps = 2;
-constexpr int kGThreads = 256;
+constexpr int kConvWarps = 4;
+constexpr int kConvThreads = 32 * kConvWarps;
+constexpr int kConvPer = static_cast<int>(kPBytes / 16) / kConvThreads;  // packed 16-byte chunks per thread
+constexpr int kMmaWarpG = 1 + kConvWarps;                                // then four epilogue warps
+constexpr int kGThreads = 32 * (kMmaWarpG + 1 + 4);
 constexpr uint32_t kGIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kGN >> 3) << 17) |
                              (static_cast<uint32_t>(kGM >> 4) << 24);  // s32 <- s8 x s8, both K-major
 constexpr size_t kGSmem = 1024 + kGStages * (kBBytes + kABytes8 + kPBytes) + 1024;
@@ -121,7 +124,7 @@ __global__ void __launch_bounds__(kGThreads, 1) w4a4_gemm_kernel(const __grid_co
   __syncthreads();
   griddep_wait();  // inputs may come from the grid before (the quantizer)
   griddep_launch_dependents();
-  if (warp == 3) {
+  if (warp == kMmaWarpG) {
     tmem_alloc(smem_u32(tmem_slot), 2 * kGN);
     tmem_relinquish();
   }
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(kGThreads, 1) w4a4_gemm_kernel(const __grid_co
     // ------------------------------------------------------------------ converters
     // Packed row m holds 64 bytes = 4 chunks of 16; chunk c gives s8 bytes [32c, 32c + 32) of the
     // K-major 128-byte row m, i.e. 16-byte slots 2c and 2c + 1, swizzled by (m & 7).
-    const int ct = threadIdx.x - 32;  // 0 .. 63
+    const int ct = threadIdx.x - 32;  // 0 .. kConvThreads - 1
     const uint32_t nib_xor = p.zero == nullptr ? 0x88888888u : 0u;
     int it = 0;
     bool ok = true;
@@ -174,12 +177,12 @@ __global__ void __launch_bounds__(kGThreads, 1) w4a4_gemm_kernel(const __grid_co
         }
         const uint4* src = reinterpret_cast<const uint4*>(pbuf + s * kPBytes);
         uint8_t* dst = abuf + s * kABytes8;
-        uint4 v[8];
+        uint4 v[kConvPer];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = src[u * 64 + ct];
+        for (int u = 0; u < kConvPer; ++u) v[u] = src[u * kConvThreads + ct];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int chunk = u * 64 + ct, m = chunk >> 2, c = chunk & 3;
+        for (int u = 0; u < kConvPer; ++u) {
+          const int chunk = u * kConvThreads + ct, m = chunk >> 2, c = chunk & 3;
           const uint2 a0 = unpack8(v[u].x ^ nib_xor), a1 = unpack8(v[u].y ^ nib_xor);
           const uint2 a2 = unpack8(v[u].z ^ nib_xor), a3 = unpack8(v[u].w ^ nib_xor);
           uint8_t* row = dst + (m >> 3) * 1024 + (m & 7) * 128;
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(kGThreads, 1) w4a4_gemm_kernel(const __grid_co
         if (lane == 0) mbar_arrive(smem_u32(&ready[s]));
       }
     }
-  } else if (warp == 3) {
+  } else if (warp == kMmaWarpG) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int it = 0, lt = 0;
@@ -276,7 +279,7 @@ __global__ void __launch_bounds__(kGThreads, 1) w4a4_gemm_kernel(const __grid_co
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 3) {
+  if (warp == kMmaWarpG) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 2 * kGN);
   }
