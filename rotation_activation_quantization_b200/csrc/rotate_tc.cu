@@ -577,6 +577,34 @@ __device__ __forceinline__ void finish_token(const float2 (&v)[kPairs], float lo
   emit_run<kPairs, kMode>(v, g, sneg, odd_neg, active, p, t, j0);
 }
 
+// ------------------------------------------------------------- the top column bit on the MMA
+//
+// Y_h = A B_0 + (-1)^h A B_1 for h = 0, 1, where B_g is the g-th column half of the staged tile
+// (kHalfBytes apart; kLbo is the tile's stride between 64-column blocks) and each Y_h has its own
+// TMEM accumulator (d_tmem + h * n_half columns): the column butterfly on the top bit, done
+// inside the fp32 accumulation. -B comes from the descriptor's negate-B bit (exact). Within each
+// accumulator, the half holding input columns 0 .. half - 1 (g_first) goes first at every K
+// step: when the outlier permutation swaps the halves, Y_1 is then accumulated as the term by
+// term negation of its unswapped sum, and the swap stays an exact sign flip.
+template <int kKSteps, uint32_t kHalfBytes, uint32_t kLbo>
+__device__ __forceinline__ void fold_mmas(uint32_t d_tmem, uint32_t n_half, uint32_t a_base, uint32_t b_base,
+                                          int g_first, uint32_t idesc) {
+  constexpr uint32_t kNegB = 1u << 14;
+  const uint32_t b_first = b_base + static_cast<uint32_t>(g_first) * kHalfBytes;
+  const uint32_t b_second = b_base + static_cast<uint32_t>(g_first ^ 1) * kHalfBytes;
+  const uint32_t id_first1 = g_first ? idesc | kNegB : idesc, id_second1 = g_first ? idesc : idesc | kNegB;
+#pragma unroll
+  for (int ks = 0; ks < kKSteps; ++ks) {
+    const uint64_t ad = smem_desc(a_base + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+    const uint64_t b0 = smem_desc(b_first + ks * 2048, kLbo, 1024);
+    const uint64_t b1 = smem_desc(b_second + ks * 2048, kLbo, 1024);
+    mma_bf16(d_tmem, ad, b0, idesc, ks > 0 ? 1u : 0u);
+    mma_bf16(d_tmem, ad, b1, idesc, 1u);
+    mma_bf16(d_tmem + n_half, ad, b0, id_first1, ks > 0 ? 1u : 0u);
+    mma_bf16(d_tmem + n_half, ad, b1, id_second1, 1u);
+  }
+}
+
 // ------------------------------------------------------------------------------------- kernel
 
 // ------------------------------------------------------------- streamed variant (<= 128 columns)
@@ -994,11 +1022,12 @@ __global__ void __launch_bounds__(stream_threads(kNcol), 1) rotq_stream_kernel(T
 // into the swizzled MMA tile (three stages fit beside A), and two D warps convert each stage in
 // place: sign flips, the word permutation, and the permutation of the 16-byte slots inside each
 // 128-byte row (column bits 3-5; bits 6-7 pick the TMA box, bit 0 is folded into the epilogue).
-// One N = 256 MMA chain per token writes Z = [Z0 | Z1] (input columns 0..127 | 128..255) to TMEM.
-// Eight epilogue warps share a token: the warp for half h and lane quadrant q forms
-// Y_h = Z0 + (-1)^h Z1 -- the column butterfly on bit 7 -- 16 columns at a time, then runs the
-// remaining seven butterfly stages, min/max, the 8-warp exchange and quantization on its 128
-// values. (A token's 28,672-32,768 fp32 values fill the register file, so two tokens' epilogues
+// The column butterfly on bit 7 runs on the tensor cores too: two N = 128 MMA chains per token,
+// each accumulating over both 128-column halves of the tile, write Y_0 = A X_0 + A X_1 and
+// Y_1 = A X_0 - A X_1 to TMEM (twice the MMA work of one N = 256 chain, which the tensor pipe has
+// to spare, for one fewer add per value and a single TMEM load per thread). Eight epilogue
+// warps share a token: the warp for half h and lane quadrant q loads its 128 values of Y_h, then
+// runs the remaining seven butterfly stages, min/max, the 8-warp exchange and quantization. (A token's 28,672-32,768 fp32 values fill the register file, so two tokens' epilogues
 // cannot overlap here; a version with two groups of four warps on alternate tokens, each parking
 // half of its 256-column line in TMEM, held the TMEM buffer through the whole epilogue and ran
 // slower: 40 % of the HBM roofline against 50 % at n = 28672.)
@@ -1056,7 +1085,7 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
   static_assert(kStageChunks % kDT == 0, "D lanes own whole chunks");
   constexpr int kDBatch = 4;
   constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
-                              (static_cast<uint32_t>(kNcol >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+                              (static_cast<uint32_t>(kHalf >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
   constexpr int kDWarp0 = kWideEpiWarps;
   constexpr int kTmaWarp = kDWarp0 + kWideDWarps;
   constexpr int kMmaWarp = kTmaWarp + 1;
@@ -1175,6 +1204,7 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t a_base = smem_u32(a_smem);
+      const int g_first = box_xor >> 1;  // the tile half that holds input columns 0..127
       int i = 0;
       for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++i) {
         const int st = i % S, tb = i % kTBufs;
@@ -1184,14 +1214,10 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + tb * kNcol;
         const uint32_t b_base = smem_u32(ring + st * kStageBytes);
-#pragma unroll
-        for (int ks = 0; ks < kKSteps; ++ks) {
-          const uint64_t ad = smem_desc(a_base + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc(b_base + ks * 2048, kChunkBytes, 1024);
-          mma_bf16(d_tmem, ad, bd, kIdesc, ks > 0 ? 1u : 0u);
-        }
+        // Y_h = A B_0 + (-1)^h A B_1 (B_g = tile columns 128g .. 128g + 127), see fold_mmas
+        fold_mmas<kKSteps, 2 * kChunkBytes, kChunkBytes>(tmem_base + tb * kNcol, kHalf, a_base, b_base, g_first,
+                                                          kIdesc);
         mma_commit(smem_u32(&empty[st]));
         mma_commit(smem_u32(&tfull[tb]));
       }
@@ -1245,21 +1271,9 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
         continue;
       }
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tb * kNcol;
-      // Y_h = Z0 + (-1)^h Z1, sixteen columns at a time. When the outlier permutation swaps the
-      // halves (bit 7) this gives Z1 + Z0 and Z1 - Z0 = -(Z0 - Z1): bit for bit the sign-adjusted
-      // values, as with the other permutation bits.
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tb * kNcol + half * kHalf;
       float2 v[kPairs];
-#pragma unroll
-      for (int c = 0; c < kHalf; c += 16) {
-        uint32_t r1[16];
-        tmem_ld16_pair(taddr + c, taddr + kHalf + c, v + c / 2, r1);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float2 z1 = make_float2(__uint_as_float(r1[2 * k]), __uint_as_float(r1[2 * k + 1]));
-          v[c / 2 + k] = half ? fsub2(v[c / 2 + k], z1) : __fadd2_rn(v[c / 2 + k], z1);
-        }
-      }
+      tmem_load_pairs<0, kPairs, kPairs>(taddr, v);  // Y_half: one 128-column load, one wait
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[tb]));

@@ -189,20 +189,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       ::"r"(taddr), SIGNROT_W8(0), SIGNROT_W8(8), SIGNROT_W8(16), SIGNROT_W8(24)
       : "memory");
 }
-// Two 32-lane x 16-column loads, one wait: columns [a0, a0 + 16) into the pairs z[0..8) and
-// [a1, a1 + 16) into r.
-__device__ __forceinline__ void tmem_ld16_pair(uint32_t a0, uint32_t a1, float2* z, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n"
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,"
-      "%31}, [%33];\n"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=f"(z[0].x), "=f"(z[0].y), "=f"(z[1].x), "=f"(z[1].y), "=f"(z[2].x), "=f"(z[2].y), "=f"(z[3].x),
-        "=f"(z[3].y), "=f"(z[4].x), "=f"(z[4].y), "=f"(z[5].x), "=f"(z[5].y), "=f"(z[6].x), "=f"(z[6].y),
-        "=f"(z[7].x), "=f"(z[7].y), SIGNROT_R8(0), SIGNROT_R8(8)
-      : "r"(a0), "r"(a1)
-      : "memory");
-}
 #undef SIGNROT_R8
 #undef SIGNROT_W8
 
