@@ -158,10 +158,13 @@ signrot_status signrot_rotate_quant(const void* x, int32_t dtype, int64_t T, int
  * adjustment given by its outlier channel instead of a materialised s: k[0] (int32, device) and
  * x_k = xk[0] (float, device), as written by signrot_calibrate. The result equals calling
  * signrot_rotate(_quant) with s = signrot_build_sign(n, k, xk, d), bit for bit on the fused
- * kernels for n >= 7168 (F = 28) or n >= 8192. For the short rows n = 3584 and 4096 the outlier
- * form runs a kernel that tiles four tokens per tensor-core tile and keeps channel k out of its
- * fp32 sums (adding its exact contribution once at the end), while a sign vector takes the exact
- * generic kernel; both give the formula's codes except at rounding ties. Because
+ * kernels for n >= 7168 (F = 28) or n >= 8192. For the short rows n = 3584 and 4096 (bf16) the
+ * outlier form runs a kernel that tiles four tokens per tensor-core tile, keeping channel k out
+ * of its fp32 sums and adding its exact contribution once at the end; for n = 512, 1024 and 2048
+ * (fp32 or bf16, rows 16-byte aligned) it runs one that gives each token one warp and fp64 sums.
+ * A sign vector takes the exact generic kernel on these shapes; all give the formula's codes
+ * except at rounding ties.
+ * Because
  * s_j = sgn(H[j][k] D_k x_k) is a signed column of H, it factorises along the
  * Kronecker structure and is folded into the rotation itself, so the sign adjustment costs no
  * per-element work (the explainer's "at inference the only new work is an element-wise sign

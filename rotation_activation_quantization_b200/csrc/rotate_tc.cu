@@ -1318,6 +1318,114 @@ __global__ void __launch_bounds__(kWideThreads, 1) rotq_wide_kernel(const __grid
   }
 }
 
+// ------------------------------------------------------------- short rows: one warp per token
+//
+// n = 512, 1024, 2048 (F = 1), fp32 or bf16 rows, s in its outlier form (BASELINE config C1:
+// n = 1024, fp32, a massive outlier on every token). One warp per token: lane l holds channels
+// [l V, l V + V) (V = n / 32); the low log2(V) Walsh stages run in the lane's registers, the five
+// high ones across lanes (shfl.xor). The sums are fp64 and y = s w / sqrt(n) is rounded once to
+// fp32, so y is the correctly rounded fp32 of the exact rotation up to a rare double rounding.
+// That matters for the token's extremes: on rows like C1's every output sits near
+// |x_k| / sqrt(n) with a spread of ~1, so |y| / scale reaches ~700, and an extreme one ulp off
+// (what fp32 sums give) moves the scale by ~5e-6 and every code by ~3e-3 of a step -- past the
+// rounding-tie window on ~1 % of the elements. With fp64 sums the scale is the oracle's.
+constexpr int kSmallWarps = 4;
+
+template <int kV, bool kF32In, int kMode>
+__global__ void __launch_bounds__(32 * kSmallWarps) rotq_small_kernel(TcParams p) {
+  static_assert(kV == 16 || kV == 32 || kV == 64, "512, 1024 or 2048 channels");
+  constexpr int kPairs = kV / 2;
+  const int lane = threadIdx.x & 31;
+  const int gw = static_cast<int>(blockIdx.x) * kSmallWarps + static_cast<int>(threadIdx.x >> 5);
+  const int nw = static_cast<int>(gridDim.x) * kSmallWarps;
+  griddep_wait();  // inputs may come from the grid before
+  griddep_launch_dependents();
+  const OutlierRef o = load_outlier(p);
+  const int k = o.k;
+  if (p.kp != nullptr && (k < 0 || k >= p.n)) flag_error(2u);  // not a channel: no sign adjustment
+  const bool pattern = p.kp != nullptr && k >= 0 && k < p.n && o.xk != 0.f;
+  const int j0 = lane * kV;
+  // D of this lane's channels, and s with 1/sqrt(n) folded in (s_j = sgn(H[j,k] D_k x_k) =
+  // (-1)^popcount(j & k) sgn(D_k) sgn(x_k))
+  uint64_t dbits = 0, sbits = 0;
+#pragma unroll
+  for (int v = 0; v < kV; ++v)
+    if (p.d[j0 + v] < 0) dbits |= 1ull << v;
+  if (pattern) {
+    const uint32_t sig = ((o.xk < 0.f) != (p.d[k] < 0)) ? 1u : 0u;
+#pragma unroll
+    for (int v = 0; v < kV; ++v)
+      if (((__popc(static_cast<uint32_t>((j0 + v) & k)) & 1u) ^ sig) != 0u) sbits |= 1ull << v;
+  }
+  const double rs = 1.0 / sqrt(static_cast<double>(p.n));
+
+  for (int t = gw; t < p.T; t += nw) {
+    double a[kV];
+    if constexpr (kF32In) {
+      const float4* xr = reinterpret_cast<const float4*>(static_cast<const float*>(p.xraw) +
+                                                         static_cast<int64_t>(t) * p.ldx + j0);
+#pragma unroll
+      for (int i = 0; i < kV / 4; ++i) {
+        const float4 f = xr[i];
+        a[4 * i] = f.x;
+        a[4 * i + 1] = f.y;
+        a[4 * i + 2] = f.z;
+        a[4 * i + 3] = f.w;
+      }
+    } else {
+      const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.xraw) +
+                                                       static_cast<int64_t>(t) * p.ldx + j0);
+#pragma unroll
+      for (int i = 0; i < kV / 8; ++i) {
+        const uint4 w = xr[i];
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          a[8 * i + 2 * e] = __uint_as_float(u[e] << 16);
+          a[8 * i + 2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
+        }
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < kV; ++v)  // x' = D x
+      if ((dbits >> v) & 1ull) a[v] = -a[v];
+    // the stages on the lane-local bits of j
+#pragma unroll
+    for (int h = 1; h < kV; h <<= 1) {
+#pragma unroll
+      for (int v = 0; v < kV; ++v) {
+        if ((v & h) == 0) {
+          const double u = a[v], w = a[v + h];
+          a[v] = u + w;
+          a[v + h] = u - w;
+        }
+      }
+    }
+    // the stages on the lane bits: the lower lane keeps u + w, the upper one u - w
+#pragma unroll
+    for (int b = 0; b < 5; ++b) {
+      const bool upper = (lane >> b) & 1;
+#pragma unroll
+      for (int v = 0; v < kV; ++v) {
+        const double w = __shfl_xor_sync(0xffffffffu, a[v], 1 << b);
+        a[v] = upper ? w - a[v] : a[v] + w;
+      }
+    }
+    // y = s w / sqrt(n), rounded once to fp32
+    float2 y[kPairs];
+#pragma unroll
+    for (int i = 0; i < kPairs; ++i) {
+      const double y0 = ((sbits >> (2 * i)) & 1ull) ? -a[2 * i] * rs : a[2 * i] * rs;
+      const double y1 = ((sbits >> (2 * i + 1)) & 1ull) ? -a[2 * i + 1] * rs : a[2 * i + 1] * rs;
+      y[i] = make_float2(__double2float_rn(y0), __double2float_rn(y1));
+    }
+    float lx, hx, ly, hy;
+    local_minmax_xy<kPairs>(y, lx, hx, ly, hy);
+    const float lo = warp_min(fminf(lx, ly)), hi = warp_max(fmaxf(hx, hy));
+    finish_token<kPairs, kMode>(y, lo, hi, false, false, true, lane == 0, p, t, j0);  // p.inv_sqrt_n = 1
+  }
+}
+
 // ------------------------------------------------------------------------------------- host
 
 // Per kernel instantiation: its shared-memory attribute, set once per device, and the device's SM
@@ -1445,9 +1553,72 @@ cudaError_t dispatch_stream(const TcParams& p, bool vec_sign, int mode, cudaStre
 
 }  // namespace
 
+template <int kV, bool kF32In>
+cudaError_t launch_small_mode(const TcParams& p, int mode, cudaStream_t st) {
+  const void* kerns[5] = {reinterpret_cast<const void*>(rotq_small_kernel<kV, kF32In, kModeY>),
+                          reinterpret_cast<const void*>(rotq_small_kernel<kV, kF32In, kModeA4>),
+                          reinterpret_cast<const void*>(rotq_small_kernel<kV, kF32In, kModeA8>),
+                          reinterpret_cast<const void*>(rotq_small_kernel<kV, kF32In, kModeS4>),
+                          reinterpret_cast<const void*>(rotq_small_kernel<kV, kF32In, kModeS8>)};
+  static KernelSetup setup[5];
+  int sms = 0;
+  cudaError_t e = setup[mode].prepare(kerns[mode], 0, &sms);
+  if (e != cudaSuccess) return e;
+  const int64_t ctas = (static_cast<int64_t>(p.T) + kSmallWarps - 1) / kSmallWarps;
+  const int grid = static_cast<int>(ctas < 16LL * sms ? ctas : 16LL * sms);
+  switch (mode) {
+    case kModeY: e = launch_pdl(rotq_small_kernel<kV, kF32In, kModeY>, grid, 32 * kSmallWarps, 0, st, p); break;
+    case kModeA4: e = launch_pdl(rotq_small_kernel<kV, kF32In, kModeA4>, grid, 32 * kSmallWarps, 0, st, p); break;
+    case kModeA8: e = launch_pdl(rotq_small_kernel<kV, kF32In, kModeA8>, grid, 32 * kSmallWarps, 0, st, p); break;
+    case kModeS4: e = launch_pdl(rotq_small_kernel<kV, kF32In, kModeS4>, grid, 32 * kSmallWarps, 0, st, p); break;
+    default: e = launch_pdl(rotq_small_kernel<kV, kF32In, kModeS8>, grid, 32 * kSmallWarps, 0, st, p); break;
+  }
+  count_launch();
+  return e;
+}
+
+// Rows of 512-2048 channels (F = 1) with s in its outlier form: one warp per token.
+cudaError_t launch_small(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
+  const bool f32 = a.dtype == kF32;
+  const int es = f32 ? 4 : 2;
+  if (reinterpret_cast<uintptr_t>(a.x) % 16 != 0 || (a.ld * es) % 16 != 0) return cudaErrorNotSupported;
+  const bool quant = a.q != nullptr;
+  const int mode = !quant ? kModeY : (a.sym ? (a.bits == 8 ? kModeS8 : kModeS4) : (a.bits == 8 ? kModeA8 : kModeA4));
+  if (quant && reinterpret_cast<uintptr_t>(a.q) % 16 != 0) return cudaErrorNotSupported;
+  if (!quant && (reinterpret_cast<uintptr_t>(a.y) % 16 != 0 || a.ldy % 4 != 0)) return cudaErrorNotSupported;
+  TcParams p{};
+  p.xraw = a.x;
+  p.ldx = a.ld;
+  p.T = static_cast<int32_t>(a.T);
+  p.n = a.shape.n;
+  p.logM = a.shape.logM;
+  p.d = a.d;
+  p.s = nullptr;
+  p.kp = a.kp;
+  p.xkp = a.xkp;
+  p.q = a.q;
+  p.scale = a.scale;
+  p.zero = a.zero;
+  p.y = a.y;
+  p.ldy = a.ldy;
+  p.clip = a.clip;
+  p.inv_sqrt_n = 1.f;  // the kernel stores y = s w / sqrt(n) itself: the grid's multiplier is 1
+  p.h = h;
+  switch (a.shape.n) {
+    case 512: return f32 ? launch_small_mode<16, true>(p, mode, st) : launch_small_mode<16, false>(p, mode, st);
+    case 1024: return f32 ? launch_small_mode<32, true>(p, mode, st) : launch_small_mode<32, false>(p, mode, st);
+    default: return f32 ? launch_small_mode<64, true>(p, mode, st) : launch_small_mode<64, false>(p, mode, st);
+  }
+}
+
 constexpr bool kShortRowTiles = true;
 
 cudaError_t launch_rotate_fast(const RotateArgs& a, const H28Masks& h, cudaStream_t st) {
+  if (a.T > 0 && a.T <= 0x7fffffff && a.shape.F == 1 && a.kp != nullptr &&
+      (a.shape.n == 512 || a.shape.n == 1024 || a.shape.n == 2048)) {
+    cudaError_t e = launch_small(a, h, st);
+    if (e != cudaErrorNotSupported) return e;
+  }
   if (a.dtype != kBF16 || a.T <= 0 || a.T > 0x7fffffff) return cudaErrorNotSupported;
   if (a.shape.F != 1 && a.shape.F != 28) return cudaErrorNotSupported;
   const bool f28 = a.shape.F == 28;

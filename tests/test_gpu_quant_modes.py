@@ -1,8 +1,9 @@
 """GPU tests of the quantizer variants: the asymmetric grid with 8 bits (codes 0..255, one per
 byte) and the symmetric grid with 4 and 8 bits (codes -7..7 as two's-complement nibbles, -127..127
 as int8; scale = max|y| / L, no zero-point), on the fused kernels (n = 28 * {256, 512, 1024},
-16384) and the generic kernel (n = 1024, 4096; fp32 and bf16 rows), against the float64 oracle.
-The outlier-channel entry points must give the same bits as the materialised sign vector."""
+16384), the generic kernel (the sign-vector entry at n = 1024 fp32 and 4096) and the short-row
+kernels (the outlier entry there), against the float64 oracle. Where both entries run the same
+kernel they must give the same bits."""
 import numpy as np
 import pytest
 
@@ -51,8 +52,9 @@ def test_quantizer_variants(sr, n, dtype):
     s_ref = oracle_sign(x64, d)
     assert (s_t.cpu().numpy() == s_ref).all()
     y_ref = o.rotate(x64, d, s_ref)
-    # on the short rows (n = 3584, 4096) the two entries run different kernels: each is checked
-    same_kernel = not (dtype == "bf16" and n in (3584, 4096))
+    # on the short rows (n = 3584, 4096 bf16; n = 512 .. 2048) the two entries run different
+    # kernels: each is checked against the oracle
+    same_kernel = not ((dtype == "bf16" and n in (3584, 4096)) or n in (512, 1024, 2048))
     for bits, sym in MODES:
         if sym:
             q1, sc1 = sr.rotate_quant_sym(x_t, d_t, s_t, bits=bits)
