@@ -108,3 +108,30 @@ def test_scale_bar_is_not_widened_on_long_outlier_rows():
     bad[5] *= 1 + 3e-5
     with pytest.raises(AssertionError):
         check_quant(encode(codes, 4, False), bad, zero, y, x64=x64)
+
+
+def test_an_extreme_one_ulp_off_fails_on_outlier_dominated_rows():
+    """Rows like BASELINE config C1 (n = 1024 fp32, a massive outlier on every token): after the
+    sign adjustment every output sits near |x_k| / sqrt(n) with a spread of about one, so
+    |y| / scale is ~700. A grid built from a maximum one fp32 ulp above the true one passes the
+    1e-5 scale bar, yet it moves every code by ~3e-3 of a step, and the checker rejects the codes.
+    This is why the one-warp kernel for these rows sums in fp64."""
+    rng = np.random.default_rng(11)
+    n, T, k = 1024, 16, 300
+    x = rng.normal(0.0, 0.3, size=(T, n)).astype(np.float32)
+    x[:, k] = (np.where(rng.random(T) < 0.5, -1.0, 1.0) * rng.uniform(1000.0, 2000.0, size=T)).astype(np.float32)
+    d = np.where(rng.random(n) < 0.5, -1, 1).astype(np.int8)
+    x64 = x.astype(np.float64)
+    kk, xk = o.calibrate(x64)
+    y = o.rotate_fast(x64, d, o.build_sign(n, kk, xk, d))
+    y32 = y.astype(np.float32)
+    lo = y32.min(axis=1)
+    hi = np.nextafter(y32.max(axis=1), np.float32(np.inf))
+    scale = ((hi - lo) / np.float32(15)).astype(np.float32)
+    zero = np.rint(-lo / scale).astype(np.float32)
+    codes = np.clip(np.rint(y32 / scale[:, None]) + zero[:, None], 0, 15).astype(np.uint8)
+    _, scale_ref, _ = o.quantize_asym(y)
+    assert (np.abs(scale.astype(np.float64) / scale_ref - 1) <= 1e-5).all()
+    assert float(np.median(np.abs(y32).max(axis=1) / scale_ref)) > 300
+    with pytest.raises(AssertionError):
+        check_quant(encode(codes, 4, False), scale, zero, y, x64=x64)
