@@ -1,38 +1,40 @@
-// Fused rotate + sign-adjust + asymmetric INT4 quantization on B200 tensor cores (tcgen05 + TMEM).
+// Fused rotate + sign-adjust + per-token quantization on B200 tensor cores (tcgen05 + TMEM), and a
+// one-warp-per-token kernel for rows of 512-2048 channels.
 //
 // What one token row computes (SignRot abstract and explainer, "The standard fix is rotation" and
 // "SignRot asks one crowd to walk across the hall"): y = diag(s) H diag(D) x / sqrt(n), then the
-// per-token asymmetric 4-bit grid ("Picture the photographer", "Worked example").
+// per-token asymmetric 4-bit grid ("Picture the photographer", "Worked example") or one of its
+// variants (8 bits, symmetric).
 //
 // How it maps onto the hardware. Write the channel index as j = (a, h2, b) with n = 28 * M,
 // a in [0, 28), h2 in [0, 4) (top two bits of the length-M axis) and b in [0, M/4), or for
 // power-of-two n as j = (r, b) with r in [0, 128). The rotation factors as
 //     H = (H_28 kron H_4) kron H_{M/4}      (or H_128 kron H_{n/128})
 // and the first factor is a dense 112 x 112 (128 x 128) block with entries +/-1. It is applied as
-// one tcgen05 MMA chain per token on the exact bf16 inputs (+/-1 times bf16 is exact; fp32
+// a tcgen05 MMA chain per token on the exact bf16 inputs (+/-1 times bf16 is exact; fp32
 // accumulation):
 //     A  = rowsign (.) (H_28 kron H_4), 128 x 128 bf16, K-major, SMEM (built once per CTA)
-//     B  = D (.) x viewed as [K = (c, h2) rows][N = b columns], bf16, MN-major, SMEM (TMA tiles)
+//     B  = D (.) x viewed as [K = (c, h2) rows][N = b columns], bf16, MN-major, SMEM
 //     Dt = A B in TMEM: lane = (h2', a) row, column = b.
-// Each TMEM lane is then one length-M/4 line of the remaining Walsh-Hadamard factor, so every
-// remaining FWHT stage runs inside one thread's registers, and each thread ends up owning a
-// contiguous run of output channels (contiguous packed INT4 stores). The per-token min/max is a
-// warp reduction plus a 4-warp exchange through shared memory.
+// Each TMEM lane is then one length-M/4 line of the remaining Walsh-Hadamard factor, so the
+// remaining FWHT stages run inside one thread's registers (for 256-column lines the stage on the
+// top column bit runs inside the MMA accumulation instead), and each thread ends up owning a
+// contiguous run of output channels (contiguous packed stores). The per-token min/max is a warp
+// reduction plus an exchange between the token's warps through shared memory.
 //
-// Sign vector from an outlier channel k (signrot_build_sign's form, s_j = sgn(H[j,k] D_k x_k))
-// costs nothing here: with k = (c_k, h2_k, e) the sign factorises into sigma * H_28[a][c_k] *
-// (-1)^popcount(h2 & h2_k) (folded into A's rows) times (-1)^popcount(b & e), which is folded
-// into the FWHT butterflies by swapping the subtraction's operands on the stages whose bit of e
-// is set. A general s vector is applied elementwise in the epilogue instead.
+// A sign vector from an outlier channel k (signrot_build_sign's form, s_j = sgn(H[j,k] D_k x_k))
+// costs nothing per element: s = sigma * H_28[a][c_k] * (-1)^popcount(hi & e_hi) *
+// (-1)^popcount(b & e_lo). The row part is folded into A's rows; the column part becomes a
+// permutation of the input columns, b -> b ^ e_lo (the TMA box order, and the 16-byte slots and
+// words the D pass moves), except its bit 0, which the epilogue applies as a sign on the odd
+// columns; sigma is a sign on every output. A general s vector is applied elementwise in the
+// epilogue instead.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over tokens):
-//   warps 0-3  epilogue: TMEM -> registers, FWHT, min/max, quantize, pack, store (TMEM lane
-//              quadrant = warp index)
-//   warps 4-7  D pass: flip the sign bits of the staged bf16 tile in shared memory
-//   warp 8     TMA producer (one elected lane)
-//   warp 9     TMEM allocator and MMA issuer (one elected lane)
-// Pipeline: TMA -> full[s] -> D pass -> dready[s] -> MMA -> (empty[s], tfull[b]) -> epilogue ->
-// tempty[b] -> MMA. Shared-memory stages form a ring; TMEM holds two token accumulators.
+// Kernels (each one's own comment gives its warp roles and pipeline):
+//   rotq_stream_kernel  64-128 columns per TMEM lane (n = 7168 .. 14336, 8192 .. 16384), and the
+//                       short rows n = 3584, 4096 with four tokens to a 128-column tile
+//   rotq_wide_kernel    256 columns per TMEM lane (n = 28672, 32768)
+//   rotq_small_kernel   n = 512, 1024, 2048 (F = 1) with s in its outlier form: one warp per token
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
